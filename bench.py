@@ -1,0 +1,390 @@
+"""Benchmark: verified draft-tree nodes per second through a gated-delta linear-attention
+layer on B200, and the achieved fraction of the HBM roofline.
+
+One step = the whole hot path over one batch: tree_verify (metadata, S_root products,
+tree solve, outputs) followed by tree_commit of every sequence's accepted path.  The
+workload is 32 sequences x 32 heads of 64-node draft trees (depth <= 8, branching 1..4),
+dk = dv = 128, bf16 q/k/v, fp32 S_root and gates.  One node = one tree node of one
+sequence processed for all heads.  Inputs are rotated over three seeded sets (3 x 168 MB
+of verify traffic, larger than the 126 MB L2), so every step reads cold HBM.
+
+Usage:
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+Multi-GPU (one process per GPU under torchrun): each rank runs an independent replica
+of the workload on its own GPU; no collective touches the data path, only a barrier and
+a max-reduction of the timings.  value = nodes processed by all ranks / max rank time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "verified tree nodes/sec (GDN, dk=dv=128) at 1 B200; % of HBM roofline"
+WORKLOAD_IDX = 3
+WORKLOAD = "gdn draft trees B=32 H=32 nodes=64 depth<=8 branching<=4 dk=dv=128 bf16 qkv fp32 state"
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+N_SETS = 3
+
+
+# ----------------------------------------------------------------------------- byte counts
+def verify_bytes(w) -> int:
+    """Algorithmic bytes of one tree_verify: inputs read once, outputs written once."""
+    in_b = 2 if w.in_dtype == "bf16" else 4
+    out_b = 2 if w.out_dtype == "bf16" else 4
+    T, H, B = w.T, w.H, w.B
+    return (B * H * w.dk * w.dv * 4 + T * H * (2 * w.dk + w.dv) * in_b + T * H * 8 +
+            4 * T + 4 * (B + 1) + T * H * w.dv * out_b + T * H * w.dv * 4)
+
+
+def commit_bytes(w) -> int:
+    """Algorithmic bytes of one tree_commit: S_root read + S_new written + path rows."""
+    in_b = 2 if w.in_dtype == "bf16" else 4
+    m = int((w.accepted_path >= 0).sum())
+    return (2 * w.B * w.H * w.dk * w.dv * 4 + m * w.H * (w.dv * 4 + w.dk * in_b + 4) +
+            w.accepted_path.size * 4 + 4 * (w.B + 1) + 4 * m)
+
+
+# ---------------------------------------------------------------------------- distributed
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity on one rank)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(nodes_per_rank_step: int, steps: int, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: every rank's nodes over the slowest rank's time."""
+    return nodes_per_rank_step * steps * world / max_seconds
+
+
+# ---------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.samples = []
+        self._stop = threading.Event()
+        self._thread = None
+
+    def _one(self):
+        try:
+            out = subprocess.run(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                  "--format=csv,noheader,nounits"], capture_output=True,
+                                 text=True, timeout=5).stdout.strip()
+            if out:
+                self.samples.append([x.strip() for x in out.split(",")])
+        except Exception:
+            pass
+
+    def _loop(self):
+        while not self._stop.is_set():
+            self._one()
+            self._stop.wait(0.2)
+
+    def start(self):
+        self._thread = threading.Thread(target=self._loop, daemon=True)
+        self._thread.start()
+
+    def stop(self) -> dict:
+        self._stop.set()
+        if self._thread:
+            self._thread.join(timeout=10)
+        if not self.samples:
+            self._one()
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4)
+                          if len(s) > 5 + i and s[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------------- peaks
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_record(kernel_file: str, kernel_name: str):
+    """Per-launch DRAM bytes from a committed ncu summary, if taken on this kernel source."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    src = os.path.join(ROOT, "linear_attention_tree_b200", "csrc", kernel_file)
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel_name)
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        if rec and rec.get("source_sha") == sha:
+            return rec.get("bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+# ------------------------------------------------------------------------------ oracle leg
+def oracle_nodes(w, rows):
+    """Time the float64 oracle on global node rows (every head of each row), plus the
+    commit of every sequence whose last node is among them.  Returns (nodes, seconds)."""
+    from threadpoolctl import threadpool_limits
+    from oracle import oracle as O
+    seq_of = np.searchsorted(w.node_offsets, np.asarray(rows), side="right") - 1
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        for row, s in zip(rows, seq_of):
+            n = int(row - w.node_offsets[s])
+            for h in range(w.H):
+                O.verify_node(w, int(s), n, h)
+            if row == w.node_offsets[s + 1] - 1:
+                for h in range(w.H):
+                    O.commit_sequence(w, int(s), h, w.accepted_path[s])
+        dt = time.perf_counter() - t0
+    return len(rows), dt
+
+
+def run_reference(args, w):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    # about two minutes of oracle work for the whole run, at least one node per step
+    per_node_s = 0.035
+    k = int(min(w.T, max(1, 120.0 / ((args.steps + args.warmup) * per_node_s))))
+    for i in range(args.warmup):
+        oracle_nodes(w, [(i * k + j) % w.T for j in range(k)])
+    total_nodes, total_t = 0, 0.0
+    for i in range(args.steps):
+        n, dt = oracle_nodes(w, [((args.warmup + i) * k + j) % w.T for j in range(k)])
+        total_nodes += n
+        total_t += dt
+    value = total_nodes / total_t
+    sample = (f"{args.steps} step(s) of {k} consecutive node(s) x {w.H} heads of the workload "
+              f"(verify of each node, commit of each sequence completed), fp64 numpy, one BLAS thread")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "nodes/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "nodes_per_tree": 64,
+                   "dk": w.dk, "dv": w.dv, "seed": 0},
+        "cpu_baseline": {"value": value, "unit": "nodes/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "nodes/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------------- GPU leg
+def run_b200(args, workloads):
+    import torch
+    import linear_attention_tree_b200 as L
+    from linear_attention_tree_b200.tensors import to_device
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    w0 = workloads[0]
+    sets = [to_device(w, dev) for w in workloads]
+    B, H, T = w0.B, w0.H, w0.T
+    prob = L.make_problem(B, H, w0.dk, w0.dv, T, w0.max_nodes, max(w.max_path for w in workloads))
+    ws = L.new_workspace(prob, dev)
+    outs = [(torch.empty((T, H, w0.dv), dtype=torch.bfloat16, device=dev),
+             torch.empty((T, H, w0.dv), dtype=torch.float32, device=dev),
+             torch.empty_like(d["S_root"])) for d in sets]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, ev=None):
+        d, (o, U, S_new) = sets[i % N_SETS], outs[i % N_SETS]
+        if ev is not None:
+            ev[0].record(stream)
+        L.tree_verify(d["q"], d["k"], d["v"], d["log_a"], d["b"], d["parent"],
+                      d["node_offsets"], d["S_root"], max_nodes=w0.max_nodes, out=o, U=U,
+                      workspace=ws, kernel=args.kernel)
+        if ev is not None:
+            ev[1].record(stream)
+        L.tree_commit(U, d["k"], d["log_a"], d["S_root"], d["node_offsets"],
+                      d["accepted_path"], max_nodes=w0.max_nodes, S_new=S_new, workspace=ws)
+        if ev is not None:
+            ev[2].record(stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    st = L.get_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+    clocks = ClockSampler(int(visible[local]) if len(visible) > local and
+                          visible[local].strip().isdigit() else local)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(i, evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    barrier()
+    elapsed_s = t_start.elapsed_time(t_end) / 1e3
+    verify_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    commit_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    max_s = max_over_ranks(elapsed_s, world, dev)
+    value = aggregate(T, args.steps, world, max_s)
+    st = L.get_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after the timed region")
+
+    # ---- end to end through the public API: pinned host inputs in, results out
+    host = [to_device(w, "cpu", pin=True) for w in workloads]
+    h_out = [torch.empty((T, H, w0.dv), dtype=torch.bfloat16).pin_memory() for _ in range(N_SETS)]
+    h_S = [torch.empty_like(h["S_root"]).pin_memory() for h in host]
+    names = ["q", "k", "v", "log_a", "b", "parent", "node_offsets", "S_root", "accepted_path"]
+    h2d = sum(host[0][n].numel() * host[0][n].element_size() for n in names)
+    d2h = h_out[0].numel() * 2 + h_S[0].numel() * 4
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step(i):
+        h, d = host[i % N_SETS], sets[i % N_SETS]
+        o, U, S_new = outs[i % N_SETS]
+        for n in names:
+            d[n].copy_(h[n], non_blocking=True)
+        L.tree_verify(d["q"], d["k"], d["v"], d["log_a"], d["b"], d["parent"],
+                      d["node_offsets"], d["S_root"], max_nodes=w0.max_nodes, out=o, U=U,
+                      workspace=ws, kernel=args.kernel)
+        L.tree_commit(U, d["k"], d["log_a"], d["S_root"], d["node_offsets"],
+                      d["accepted_path"], max_nodes=w0.max_nodes, S_new=S_new, workspace=ws)
+        h_out[i % N_SETS].copy_(o, non_blocking=True)
+        h_S[i % N_SETS].copy_(S_new, non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
+    e2e_value = aggregate(T, e2e_steps, world, e2e_s)
+
+    if rank == 0:
+        peak, peak_src = hbm_peak()
+        vb, cb = verify_bytes(w0), commit_bytes(w0)
+        v_avg = statistics.mean(verify_ms) / 1e3
+        c_avg = statistics.mean(commit_ms) / 1e3
+        tc = args.kernel != "simt" and w0.max_nodes <= 64
+        kfile, kname = ("verify_tc.cu", "verify_tc") if tc else ("verify_simt.cu", "verify_simt")
+        achieved = vb / v_avg / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": "nodes/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * max_s / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16xbf16->f32" if tc else "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": B, "H": H, "nodes_per_tree": 64,
+                       "dk": w0.dk, "dv": w0.dv, "seeds": list(range(N_SETS)),
+                       "l2": f"{N_SETS} rotating input sets, {N_SETS}x{vb / 1e6:.0f} MB > 126 MB L2",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "kernel": kname},
+            "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
+                         "unit": "GB/s", "frac": achieved / peak, "peak_source": peak_src,
+                         "traffic": traffic_record(kfile, kname),
+                         "algorithmic_bytes_per_launch": vb,
+                         "frac_of_8TBps": achieved / NOMINAL_HBM_GBS},
+            "verify_us": 1e6 * v_avg, "commit_us": 1e6 * c_avg,
+            "verify_nodes_per_s": T / v_avg,
+            "commit_roofline": {"achieved": cb / c_avg / 1e9, "unit": "GB/s",
+                                "frac": cb / c_avg / 1e9 / peak,
+                                "algorithmic_bytes_per_launch": cb},
+            "step_bytes_per_s": (vb + cb) * args.steps / max_s / 1e9,
+            "e2e": {"value": e2e_value, "unit": "nodes/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clk,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            n, dt = oracle_nodes(workloads[0], list(range(4 * 64)))
+            line["cpu_baseline"] = {
+                "value": n / dt, "unit": "nodes/s", "cores": 1, "kind": "oracle",
+                "sample": "sequences 0-3 (4 x 64 nodes x 32 heads) of the workload, verify + "
+                          "commit, fp64 numpy, one BLAS thread", "seconds": dt}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--kernel", choices=["auto", "tc", "simt"], default="auto")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from linear_attention_tree_b200 import workloads as W
+    if args.impl == "reference":
+        return run_reference(args, W.config(WORKLOAD_IDX, 0))
+    workloads = [W.config(WORKLOAD_IDX, s) for s in range(N_SETS)]
+    return run_b200(args, workloads)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

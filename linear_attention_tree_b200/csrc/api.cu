@@ -1,0 +1,161 @@
+// C ABI entry points: argument validation, kernel choice, launches.  No allocation, no
+// synchronisation except in tv_get_status.
+#include <cstring>
+
+#include "tv_internal.cuh"
+
+#ifndef TV_HAVE_TC
+#define TV_HAVE_TC 0
+#endif
+
+namespace {
+
+using namespace tv;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape / enum checks shared by all entry points.
+tv_status check_problem(const tv_problem *p) {
+  if (!p) return TV_ERR_INVALID_ARG;
+  if (p->B < 0 || p->H < 1 || p->total_nodes < 0) return TV_ERR_INVALID_ARG;
+  if (p->max_nodes < 1) return TV_ERR_INVALID_ARG;
+  if (p->mode != TV_MODE_GDN && p->mode != TV_MODE_SCALAR_DECAY) return TV_ERR_INVALID_ARG;
+  if (p->in_dtype != TV_F32 && p->in_dtype != TV_BF16) return TV_ERR_INVALID_ARG;
+  if (p->out_dtype != TV_F32 && p->out_dtype != TV_BF16) return TV_ERR_INVALID_ARG;
+  if (p->kernel < TV_KERNEL_AUTO || p->kernel > TV_KERNEL_SIMT) return TV_ERR_INVALID_ARG;
+  if (p->dk < 1 || p->dv < 1) return TV_ERR_INVALID_ARG;
+  if (p->max_nodes > kMaxNodes) return TV_ERR_UNSUPPORTED;
+  if (p->dk % 16 || p->dv % 16 || p->dk > 128 || p->dv > 128) return TV_ERR_UNSUPPORTED;
+  if (p->in_dtype == TV_F32 && p->out_dtype == TV_BF16) return TV_ERR_UNSUPPORTED;
+  // int32 indexing of every array stays in range
+  const long long T = p->total_nodes, H = p->H;
+  if (T * H * 128 > 0x7fffffffLL || (long long)p->B * H > 0x7fffffffLL) return TV_ERR_UNSUPPORTED;
+  if (T > (long long)p->B * p->max_nodes) return TV_ERR_INVALID_ARG;
+  return TV_OK;
+}
+
+bool ptr_ok(const void *ptr) { return ptr && aligned16(ptr); }
+
+bool tc_supports(const tv_problem *p) {
+  return TV_HAVE_TC && p->in_dtype == TV_BF16 && p->dk == 128 && p->dv == 128 &&
+         p->max_nodes <= 64;
+}
+
+tv_status from_cuda(cudaError_t e) { return e == cudaSuccess ? TV_OK : TV_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t tv_version(void) { return (1 << 16) | 0; }
+
+const char *tv_status_string(tv_status s) {
+  switch (s) {
+    case TV_OK: return "ok";
+    case TV_ERR_INVALID_ARG: return "invalid argument";
+    case TV_ERR_UNSUPPORTED: return "unsupported problem";
+    case TV_ERR_BAD_TREE: return "bad tree (parent not topological or node_offsets invalid)";
+    case TV_ERR_BAD_PATH: return "bad accepted path";
+    case TV_ERR_CUDA: return "CUDA runtime error";
+    case TV_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+size_t tv_workspace_size(const tv_problem *p) {
+  return check_problem(p) == TV_OK ? kWorkspaceBytes : 0;
+}
+
+tv_status tv_tree_verify(const tv_problem *p, const void *q, const void *k, const void *v,
+                         const float *log_a, const float *b, const int32_t *parent,
+                         const int32_t *node_offsets, const float *S_root, void *out,
+                         float *U, void *workspace, size_t workspace_bytes,
+                         tv_stream_t stream) {
+  tv_status st = check_problem(p);
+  if (st != TV_OK) return st;
+  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(log_a) || !ptr_ok(parent) ||
+      !ptr_ok(node_offsets) || !ptr_ok(S_root) || !ptr_ok(out) || !ptr_ok(U) ||
+      !ptr_ok(workspace))
+    return TV_ERR_INVALID_ARG;
+  if (p->mode == TV_MODE_GDN ? !ptr_ok(b) : (b && !aligned16(b))) return TV_ERR_INVALID_ARG;
+  if (workspace_bytes < kWorkspaceBytes) return TV_ERR_INVALID_ARG;
+  bool use_tc;
+  if (p->kernel == TV_KERNEL_TC) {
+    if (!tc_supports(p)) return TV_ERR_UNSUPPORTED;
+    use_tc = true;
+  } else {
+    use_tc = p->kernel == TV_KERNEL_AUTO && tc_supports(p);
+  }
+  if (p->B == 0) return TV_OK;
+  VerifyArgs a;
+  a.q = q; a.k = k; a.v = v; a.log_a = log_a; a.b = b; a.parent = parent;
+  a.node_offsets = node_offsets; a.S_root = S_root; a.out = out; a.U = U;
+  a.ws = static_cast<int *>(workspace);
+  a.B = p->B; a.H = p->H; a.dk = p->dk; a.dv = p->dv; a.T = p->total_nodes;
+  a.max_nodes = p->max_nodes;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (use_tc) return from_cuda(launch_verify_tc(a, p->mode, p->out_dtype, s));
+  return from_cuda(launch_verify_simt(a, p->mode, p->in_dtype, p->out_dtype, s));
+}
+
+tv_status tv_tree_commit(const tv_problem *p, const float *U, const void *k,
+                         const float *log_a, const float *S_root,
+                         const int32_t *node_offsets, const int32_t *accepted_path,
+                         const int32_t *parent, float *S_new, void *workspace,
+                         size_t workspace_bytes, tv_stream_t stream) {
+  tv_status st = check_problem(p);
+  if (st != TV_OK) return st;
+  if (p->max_path < 1) return TV_ERR_INVALID_ARG;
+  if (!ptr_ok(U) || !ptr_ok(k) || !ptr_ok(log_a) || !ptr_ok(S_root) || !ptr_ok(node_offsets) ||
+      !ptr_ok(accepted_path) || !ptr_ok(S_new) || !ptr_ok(workspace))
+    return TV_ERR_INVALID_ARG;
+  if (parent && !aligned16(parent)) return TV_ERR_INVALID_ARG;
+  if (workspace_bytes < kWorkspaceBytes) return TV_ERR_INVALID_ARG;
+  // S_new either is S_root or does not overlap it
+  const size_t state_bytes = (size_t)p->B * p->H * p->dv * p->dk * sizeof(float);
+  const char *a0 = reinterpret_cast<const char *>(S_root), *b0 = reinterpret_cast<const char *>(S_new);
+  if (a0 != b0 && a0 < b0 + state_bytes && b0 < a0 + state_bytes) return TV_ERR_INVALID_ARG;
+  if (p->B == 0) return TV_OK;
+  CommitArgs a;
+  a.U = U; a.k = k; a.log_a = log_a; a.S_root = S_root; a.node_offsets = node_offsets;
+  a.accepted_path = accepted_path; a.parent = parent; a.S_new = S_new;
+  a.ws = static_cast<int *>(workspace);
+  a.B = p->B; a.H = p->H; a.dk = p->dk; a.dv = p->dv; a.T = p->total_nodes;
+  a.max_nodes = p->max_nodes; a.max_path = p->max_path;
+  return from_cuda(launch_commit(a, p->in_dtype, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tv_status tv_tree_meta(const tv_problem *p, const int32_t *parent,
+                       const int32_t *node_offsets, const float *log_a, int32_t *depth,
+                       uint64_t *anc, float *cumlog, void *workspace,
+                       size_t workspace_bytes, tv_stream_t stream) {
+  tv_status st = check_problem(p);
+  if (st != TV_OK) return st;
+  if (!ptr_ok(parent) || !ptr_ok(node_offsets) || !ptr_ok(log_a) || !ptr_ok(depth) ||
+      !ptr_ok(anc) || !ptr_ok(cumlog) || !ptr_ok(workspace))
+    return TV_ERR_INVALID_ARG;
+  if (workspace_bytes < kWorkspaceBytes) return TV_ERR_INVALID_ARG;
+  if (p->B == 0) return TV_OK;
+  MetaArgs a;
+  a.parent = parent; a.node_offsets = node_offsets; a.log_a = log_a; a.depth = depth;
+  a.anc = anc; a.cumlog = cumlog; a.ws = static_cast<int *>(workspace);
+  a.B = p->B; a.H = p->H; a.T = p->total_nodes; a.max_nodes = p->max_nodes;
+  a.anc_words = (p->max_nodes + 63) / 64;
+  return from_cuda(launch_meta(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tv_status tv_get_status(void *workspace, tv_stream_t stream) {
+  if (!ptr_ok(workspace)) return TV_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int host[2] = {0, 0};
+  if (cudaMemcpyAsync(host, workspace, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return TV_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return TV_ERR_CUDA;
+  if (host[0] != TV_OK) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(host), s) != cudaSuccess) return TV_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return TV_ERR_CUDA;
+  }
+  return static_cast<tv_status>(host[0]);
+}
+
+}  // extern "C"

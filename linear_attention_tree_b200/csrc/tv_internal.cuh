@@ -1,0 +1,72 @@
+// Internal declarations shared by the library's translation units (not installed).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/tree_verify.h"
+
+namespace tv {
+
+constexpr int kMaxNodes = 256;          // largest tree one sequence may hold
+constexpr int kAncWords = kMaxNodes / 64;
+constexpr size_t kWorkspaceBytes = 256; // status word + reserved
+
+// Workspace layout (int32 words).
+enum : int { kWsStatus = 0, kWsDetail = 1 };
+
+// Device status: the first error recorded wins; later ones are dropped.
+__device__ __forceinline__ void set_status(int *ws, int code, int detail) {
+  if (atomicCAS(ws + kWsStatus, 0, code) == 0) ws[kWsDetail] = detail;
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Everything a verify kernel needs, by value.
+struct VerifyArgs {
+  const void *q, *k, *v;
+  const float *log_a, *b;
+  const int32_t *parent, *node_offsets;
+  const float *S_root;
+  void *out;
+  float *U;
+  int *ws;
+  int B, H, dk, dv, T, max_nodes;
+};
+
+struct CommitArgs {
+  const float *U;
+  const void *k;
+  const float *log_a, *S_root;
+  const int32_t *node_offsets, *accepted_path, *parent;
+  float *S_new;
+  int *ws;
+  int B, H, dk, dv, T, max_nodes, max_path;
+};
+
+struct MetaArgs {
+  const int32_t *parent, *node_offsets;
+  const float *log_a;
+  int32_t *depth;
+  uint64_t *anc;
+  float *cumlog;
+  int *ws;
+  int B, H, T, max_nodes, anc_words;
+};
+
+// Launchers (host side); each returns cudaSuccess or the launch error.
+cudaError_t launch_verify_simt(const VerifyArgs &a, int mode, int in_dtype, int out_dtype,
+                               cudaStream_t st);
+cudaError_t launch_verify_tc(const VerifyArgs &a, int mode, int out_dtype, cudaStream_t st);
+cudaError_t launch_commit(const CommitArgs &a, int in_dtype, cudaStream_t st);
+cudaError_t launch_meta(const MetaArgs &a, cudaStream_t st);
+
+}  // namespace tv

@@ -21,14 +21,14 @@ What it computes, and where the pages state it:
   Every node is computed here by walking that path from ``S_root`` step by step: there is
   no closed form, no factorisation and no triangular solve in this file.
 * The output of node n is read from the post-update state, ``o_n = S_n q_n``.
-* Pseudo-values.  The TreeWY abstract replaces per-node snapshots by a "pseudo-value
-  matrix" without printing its formula.  Reading taken: ``u_n`` is the rank-1 factor by
+* Pseudo-values.  The TreeWY abstract replaces per-node snapshots by a pseudo-value
+  matrix without printing its formula.  Reading taken: ``u_n`` is the rank-1 factor by
   which node n's own step changes its parent's decayed state,
   ``S_n = a_n S_parent + u_n k_n^T``, i.e. ``u_n = b_n (v_n - a_n S_parent k_n)`` for the
   gated delta rule and ``u_n = v_n`` for scalar decay.
 * Commit.  The accepted state is the state at the end of the accepted root-first path
-  (worked example: only ``S_c3`` is rebuilt; Twig abstract: "reconstructs only the accepted
-  state"), again by walking the recurrence from ``S_root``.
+  (worked example: only ``S_c3`` is rebuilt; the Twig abstract rebuilds one state after
+  sampling), again by walking the recurrence from ``S_root``.
 
 Each function below is pinned by tests in ``tests/test_oracle_pins.py`` against facts the
 pages or the mathematics fix (the printed worked example, the page's closed form, sequential

@@ -1,0 +1,111 @@
+"""The C-ABI library builds, loads without a GPU, exports what the header declares, and
+rejects bad arguments synchronously (before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_attention_tree_b200 as L
+from linear_attention_tree_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"TV_API\s+[\w\s\*]*?\b(tv_\w+)\s*\(", text))
+    return names
+
+
+def test_library_builds_and_loads():
+    path = build.build()
+    assert os.path.exists(path)
+    assert L.lib()._name == binding.LIB_PATH
+
+
+def test_exports_every_declared_symbol():
+    names = _declared()
+    assert {"tv_tree_verify", "tv_tree_commit", "tv_tree_meta", "tv_workspace_size",
+            "tv_get_status"} <= names
+    for n in names:
+        assert hasattr(L.lib(), n), n
+    assert set(binding.EXPORTS) <= names
+
+
+def test_problem_layout_and_version():
+    assert ctypes.sizeof(binding.Problem) == 44
+    assert L.lib().tv_version() >> 16 == 1
+    assert binding.status_string(0) == "ok"
+
+
+def _call_verify(prob, ptrs):
+    return L.lib().tv_tree_verify(ctypes.byref(prob), *ptrs, ctypes.c_size_t(256), None)
+
+
+def _fake(n=11, misalign=None):
+    # fake device addresses: the call must fail before dereferencing anything
+    ptrs = [ctypes.c_void_p(0x10000 * (i + 1)) for i in range(n)]
+    if misalign is not None:
+        ptrs[misalign] = ctypes.c_void_p(0x10000 * (misalign + 1) + 4)
+    return ptrs
+
+
+@pytest.mark.parametrize("field,value,expect", [
+    ("H", 0, binding.TV_ERR_INVALID_ARG), ("B", -1, binding.TV_ERR_INVALID_ARG),
+    ("dk", 100, binding.TV_ERR_UNSUPPORTED), ("dv", 256, binding.TV_ERR_UNSUPPORTED),
+    ("max_nodes", 257, binding.TV_ERR_UNSUPPORTED), ("max_nodes", 0, binding.TV_ERR_INVALID_ARG),
+    ("mode", 7, binding.TV_ERR_INVALID_ARG), ("in_dtype", 5, binding.TV_ERR_INVALID_ARG),
+    ("kernel", 9, binding.TV_ERR_INVALID_ARG), ("total_nodes", 999999, binding.TV_ERR_INVALID_ARG),
+])
+def test_bad_problem_rejected(field, value, expect):
+    prob = L.make_problem(4, 2, 128, 128, 64, 16, 4)
+    setattr(prob, field, value)
+    assert _call_verify(prob, _fake()) == expect
+    if expect == binding.TV_ERR_INVALID_ARG or expect == binding.TV_ERR_UNSUPPORTED:
+        assert L.workspace_size(prob) == 0
+
+
+def test_null_and_misaligned_pointers_rejected():
+    prob = L.make_problem(4, 2, 128, 128, 64, 16, 4)
+    for i in range(11):
+        ptrs = _fake()
+        ptrs[i] = None
+        assert _call_verify(prob, ptrs) == binding.TV_ERR_INVALID_ARG, i
+        assert _call_verify(prob, _fake(misalign=i)) == binding.TV_ERR_INVALID_ARG, i
+    # workspace too small
+    assert L.lib().tv_tree_verify(ctypes.byref(prob), *_fake(), ctypes.c_size_t(8), None) == \
+        binding.TV_ERR_INVALID_ARG
+
+
+def test_tc_kernel_refuses_unsupported_shapes():
+    prob = L.make_problem(4, 2, 64, 128, 64, 16, 4, kernel="tc")
+    assert _call_verify(prob, _fake()) == binding.TV_ERR_UNSUPPORTED
+    prob = L.make_problem(4, 2, 128, 128, 64, 16, 4, in_dtype=__import__("torch").float32,
+                          kernel="tc")
+    assert _call_verify(prob, _fake()) == binding.TV_ERR_UNSUPPORTED
+
+
+def test_commit_rejects_partial_overlap():
+    prob = L.make_problem(2, 2, 16, 16, 8, 4, 3)
+    state = 2 * 2 * 16 * 16 * 4
+    ptrs = [ctypes.c_void_p(0x100000 * (i + 1)) for i in range(9)]
+    ptrs[7] = ctypes.c_void_p(ptrs[3].value + 256)     # S_new overlaps S_root, not equal
+    assert L.lib().tv_tree_commit(ctypes.byref(prob), *ptrs, ctypes.c_size_t(256), None) == \
+        binding.TV_ERR_INVALID_ARG
+    prob.max_path = 0
+    assert L.lib().tv_tree_commit(ctypes.byref(prob), *ptrs, ctypes.c_size_t(256), None) == \
+        binding.TV_ERR_INVALID_ARG
+
+
+def test_product_path_has_no_cpu_fallback():
+    """The package never imports the oracle, and its functions need the CUDA library."""
+    import linear_attention_tree_b200.binding as b
+    pkg = os.path.dirname(b.__file__)
+    for fn in os.listdir(pkg):
+        if fn.endswith(".py"):
+            assert "import oracle" not in open(os.path.join(pkg, fn)).read()
+            assert "from oracle" not in open(os.path.join(pkg, fn)).read()

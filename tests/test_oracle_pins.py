@@ -5,8 +5,8 @@ itself: the worked example printed on the Bole summary page, that page's lambda-
 closed form (exponents as its example fixes them), plain sequential decoding, special
 cases with closed forms (b = 0, the delta-rule identity, one token), a brute-force
 branch-by-branch traversal with explicit per-node snapshots, and the losslessness of the
-pseudo-value factorisation (TreeWY abstract: "tree-structured WY transform", "single
-triangular solve"), solved with a library triangular solver.  ``test_planted_mistakes``
+pseudo-value factorisation (TreeWY abstract: a tree-structured WY form whose pseudo-values
+come from one triangular solve), solved here with a library triangular solver.  ``test_planted_mistakes``
 shows that plausible slips in the oracle (a dropped term, a wrong index, a transposed
 operand, the pre-update state) each fail at least one pin.
 """

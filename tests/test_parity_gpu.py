@@ -1,0 +1,129 @@
+"""Parity of the CUDA path with the float64 oracle, element by element.
+
+Bars: max|err| <= 1e-4 * RMS(oracle tensor) for fp32 inputs, <= 2e-2 * RMS for bf16
+inputs, separately for o, U and S_new.  Small problems are compared in full; the five
+named workloads at full size are compared in full where the oracle is quick (1, 2) and on
+seeded samples of (node, head) outputs and (sequence, head) states otherwise, in the same
+launch configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+
+from linear_attention_tree_b200 import workloads as W
+from oracle import oracle as O
+from tests._gpu_util import TOL, assert_close, run
+
+pytestmark = pytest.mark.gpu
+
+
+def _full_check(w, kernel="auto", out_dtype=None):
+    res, _ = run(w, kernel=kernel, out_dtype=out_dtype)
+    o, U = O.tree_verify(w)
+    S_new = O.tree_commit(w)
+    tol = TOL[w.in_dtype]
+    assert_close(res["o"], o, tol, "o")
+    if w.mode == "gdn":
+        assert_close(res["U"], U, tol, "U")
+    else:
+        np.testing.assert_array_equal(res["U"], U)     # scalar decay: U = V exactly
+    assert_close(res["S_new"], S_new, tol, "S_new")
+
+
+def _sampled_check(w, kernel="auto", n_nodes=160, n_states=24, seed=0):
+    res, _ = run(w, kernel=kernel)
+    rng = np.random.default_rng(seed)
+    tol = TOL[w.in_dtype]
+    seqs = rng.integers(0, w.B, n_nodes)
+    got_o, want_o, got_u, want_u = [], [], [], []
+    for s in seqs:
+        n = int(rng.integers(0, w.node_offsets[s + 1] - w.node_offsets[s]))
+        h = int(rng.integers(0, w.H))
+        o, u = O.verify_node(w, int(s), n, h)
+        row = int(w.node_offsets[s]) + n
+        got_o.append(res["o"][row, h]); want_o.append(o)
+        got_u.append(res["U"][row, h]); want_u.append(u)
+    assert_close(np.array(got_o), np.array(want_o), tol, "o (sampled)")
+    assert_close(np.array(got_u), np.array(want_u), tol, "U (sampled)")
+    got_s, want_s = [], []
+    for _ in range(n_states):
+        s, h = int(rng.integers(0, w.B)), int(rng.integers(0, w.H))
+        want_s.append(O.commit_sequence(w, s, h, w.accepted_path[s]))
+        got_s.append(res["S_new"][s, h])
+    assert_close(np.array(got_s), np.array(want_s), tol, "S_new (sampled)")
+
+
+@pytest.mark.parametrize("kernel", ["auto", "simt"])
+def test_config1_worked_example(kernel):
+    _full_check(W.config(1), kernel)
+
+
+@pytest.mark.parametrize("kernel", ["auto", "simt"])
+def test_config2(kernel):
+    _full_check(W.config(2), kernel)
+
+
+@pytest.mark.parametrize("idx", [3, 4, 5])
+def test_full_size_sampled(idx):
+    _sampled_check(W.config(idx))
+
+
+@pytest.mark.parametrize("idx", [3, 4, 5])
+def test_full_size_sampled_simt(idx):
+    _sampled_check(W.config(idx), kernel="simt", n_nodes=60, n_states=8, seed=1)
+
+
+@pytest.mark.parametrize("idx,seed", [(3, 1), (3, 2), (4, 1)])
+def test_extra_seeds(idx, seed):
+    _sampled_check(W.config(idx, seed=seed), n_nodes=60, n_states=8, seed=seed)
+
+
+def _ragged(seed, counts, max_depth=8, fmax=4):
+    pars = []
+    for i, c in enumerate(counts):
+        par, _ = W.frontier_tree(seed * 100 + i, c, max_depth, fmax) if c else ([], None)
+        pars.append(par)
+    return pars
+
+
+@pytest.mark.parametrize("kernel", ["auto", "simt"])
+@pytest.mark.parametrize("counts", [[64, 37, 9], [1, 63, 64, 2], [5, 0, 17]])
+def test_ragged_small_full(kernel, counts):
+    """Several sequences, ragged node counts (incl. an empty tree), compared in full."""
+    w = W.synthetic(_ragged(len(counts), counts), H=3, dk=128, dv=128,
+                    seed=sum(counts), name="ragged")
+    _full_check(w, kernel)
+
+
+@pytest.mark.parametrize("mode", ["gdn", "scalar"])
+@pytest.mark.parametrize("dk,dv", [(16, 16), (32, 64), (128, 48), (64, 128)])
+def test_dims_f32(mode, dk, dv):
+    pars = _ragged(dk + dv, [12, 30])
+    w = W.synthetic(pars, H=2, dk=dk, dv=dv, seed=dk * dv, mode=mode, in_dtype="f32",
+                    log_a_mean=-2.0, s_std=0.1)
+    _full_check(w, "simt")
+
+
+@pytest.mark.parametrize("kernel", ["auto", "simt"])
+def test_scalar_bf16(kernel):
+    pars = _ragged(5, [40, 64])
+    w = W.synthetic(pars, H=2, dk=128, dv=128, seed=5, mode="scalar", log_a_mean=-3.0)
+    _full_check(w, kernel)
+
+
+def test_bf16_in_f32_out():
+    pars = _ragged(6, [33, 20])
+    w = W.synthetic(pars, H=2, dk=128, dv=128, seed=6)
+    _full_check(w, "auto", out_dtype="f32")
+
+
+def test_wide_tree_256_nodes():
+    pars = _ragged(7, [256], max_depth=10, fmax=8)
+    w = W.synthetic(pars, H=1, dk=128, dv=128, seed=7, log_a_mean=-6.0)
+    _full_check(w, "auto")
+
+
+def test_deep_chain_256():
+    """A 256-token chain: the tree degenerates to plain sequential decoding."""
+    w = W.synthetic([[i - 1 for i in range(256)]], H=1, dk=64, dv=64, seed=8, in_dtype="f32",
+                    log_a_mean=-5.0, s_std=0.05)
+    _full_check(w, "auto")
