@@ -5,8 +5,9 @@ One step = the whole hot path over one batch: tree_verify (metadata, S_root prod
 tree solve, outputs) followed by tree_commit of every sequence's accepted path.  The
 workload is 32 sequences x 32 heads of 64-node draft trees (depth <= 8, branching 1..4),
 dk = dv = 128, bf16 q/k/v, fp32 S_root and gates.  One node = one tree node of one
-sequence processed for all heads.  Inputs are rotated over three seeded sets (3 x 168 MB
-of verify traffic, larger than the 126 MB L2), so every step reads cold HBM.
+sequence processed for all heads.  Inputs are rotated over three seeded sets (3 x 185 MB
+of verify traffic, larger than the 126 MB L2), so every step reads cold HBM.  Outputs o
+and U are fp32.
 
 Usage:
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
@@ -33,7 +34,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "verified tree nodes/sec (GDN, dk=dv=128) at 1 B200; % of HBM roofline"
 WORKLOAD_IDX = 3
-WORKLOAD = "gdn draft trees B=32 H=32 nodes=64 depth<=8 branching<=4 dk=dv=128 bf16 qkv fp32 state"
+WORKLOAD = ("gdn draft trees B=32 H=32 nodes=64 depth<=8 branching<=4 dk=dv=128, "
+            "bf16 q/k/v, fp32 state, gates and outputs")
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
 N_SETS = 3
@@ -227,7 +229,8 @@ def run_b200(args, workloads):
     B, H, T = w0.B, w0.H, w0.T
     prob = L.make_problem(B, H, w0.dk, w0.dv, T, w0.max_nodes, max(w.max_path for w in workloads))
     ws = L.new_workspace(prob, dev)
-    outs = [(torch.empty((T, H, w0.dv), dtype=torch.bfloat16, device=dev),
+    odt = torch.float32 if w0.out_dtype == "f32" else torch.bfloat16
+    outs = [(torch.empty((T, H, w0.dv), dtype=odt, device=dev),
              torch.empty((T, H, w0.dv), dtype=torch.float32, device=dev),
              torch.empty_like(d["S_root"])) for d in sets]
     stream = torch.cuda.current_stream(dev)
@@ -285,11 +288,11 @@ def run_b200(args, workloads):
 
     # ---- end to end through the public API: pinned host inputs in, results out
     host = [to_device(w, "cpu", pin=True) for w in workloads]
-    h_out = [torch.empty((T, H, w0.dv), dtype=torch.bfloat16).pin_memory() for _ in range(N_SETS)]
+    h_out = [torch.empty((T, H, w0.dv), dtype=odt).pin_memory() for _ in range(N_SETS)]
     h_S = [torch.empty_like(h["S_root"]).pin_memory() for h in host]
     names = ["q", "k", "v", "log_a", "b", "parent", "node_offsets", "S_root", "accepted_path"]
     h2d = sum(host[0][n].numel() * host[0][n].element_size() for n in names)
-    d2h = h_out[0].numel() * 2 + h_S[0].numel() * 4
+    d2h = h_out[0].numel() * h_out[0].element_size() + h_S[0].numel() * 4
     e2e_steps = max(3, min(args.steps, 20))
 
     def e2e_step(i):

@@ -164,6 +164,10 @@ TV_API tv_status tv_tree_meta(const tv_problem *p, const int32_t *parent,
  * the last call (TV_OK if none) and clear it.  Not for the hot path. */
 TV_API tv_status tv_get_status(void *workspace, tv_stream_t stream);
 
+/* Name and description of the CUDA error behind the last TV_ERR_CUDA returned on the
+ * calling host thread ("" if there was none).  Static storage; do not free. */
+TV_API const char *tv_last_cuda_error(void);
+
 /* Static English name of a status code. */
 TV_API const char *tv_status_string(tv_status s);
 

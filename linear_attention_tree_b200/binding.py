@@ -29,13 +29,16 @@ MODE = {"gdn": 0, "scalar": 1}
 DTYPE = {torch.float32: 0, torch.bfloat16: 1}
 KERNEL = {"auto": 0, "tc": 1, "simt": 2}
 EXPORTS = ("tv_workspace_size", "tv_tree_verify", "tv_tree_commit", "tv_tree_meta",
-           "tv_get_status", "tv_status_string", "tv_version")
+           "tv_get_status", "tv_status_string", "tv_last_cuda_error", "tv_version")
 
 
 class TreeVerifyError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        detail = ""
+        if status == TV_ERR_CUDA:
+            detail = " [" + lib().tv_last_cuda_error().decode() + "]"
+        super().__init__(f"{what}: {status_string(status)} (status {status}){detail}")
 
 
 class Problem(ctypes.Structure):
@@ -69,6 +72,8 @@ def lib() -> ctypes.CDLL:
         L.tv_get_status.restype = ctypes.c_int
         L.tv_status_string.argtypes = [ctypes.c_int]
         L.tv_status_string.restype = ctypes.c_char_p
+        L.tv_last_cuda_error.argtypes = []
+        L.tv_last_cuda_error.restype = ctypes.c_char_p
         L.tv_version.argtypes = []
         L.tv_version.restype = ctypes.c_int32
         _lib = L

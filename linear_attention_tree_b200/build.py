@@ -47,7 +47,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     tmp = LIB + ".tmp"
     cmd = [nvcc_path(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared",
            "-Xcompiler", "-fPIC,-fvisibility=hidden", "-cudart", "static",
-           "-I", INCLUDE, "-DTV_HAVE_TC=1", "-o", tmp, *sources()]
+           "-I", INCLUDE, "-o", tmp, *sources()]
     if ptxas_info:
         cmd[1:1] = ["-Xptxas", "-v"]
     if verbose:

@@ -1,5 +1,6 @@
 // C ABI entry points: argument validation, kernel choice, launches.  No allocation, no
 // synchronisation except in tv_get_status.
+#include <cstdio>
 #include <cstring>
 
 #include "tv_internal.cuh"
@@ -41,13 +42,27 @@ bool tc_supports(const tv_problem *p) {
          p->max_nodes <= 64;
 }
 
-tv_status from_cuda(cudaError_t e) { return e == cudaSuccess ? TV_OK : TV_ERR_CUDA; }
+thread_local cudaError_t g_last_cuda = cudaSuccess;
+
+tv_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return TV_OK;
+  g_last_cuda = e;
+  return TV_ERR_CUDA;
+}
 
 }  // namespace
 
 extern "C" {
 
 int32_t tv_version(void) { return (1 << 16) | 0; }
+
+const char *tv_last_cuda_error(void) {
+  if (g_last_cuda == cudaSuccess) return "";
+  static thread_local char buf[256];
+  snprintf(buf, sizeof(buf), "%s: %s", cudaGetErrorName(g_last_cuda),
+           cudaGetErrorString(g_last_cuda));
+  return buf;
+}
 
 const char *tv_status_string(tv_status s) {
   switch (s) {
@@ -106,6 +121,7 @@ tv_status tv_tree_commit(const tv_problem *p, const float *U, const void *k,
   tv_status st = check_problem(p);
   if (st != TV_OK) return st;
   if (p->max_path < 1) return TV_ERR_INVALID_ARG;
+  if (p->max_path > commit_max_path_width()) return TV_ERR_UNSUPPORTED;
   if (!ptr_ok(U) || !ptr_ok(k) || !ptr_ok(log_a) || !ptr_ok(S_root) || !ptr_ok(node_offsets) ||
       !ptr_ok(accepted_path) || !ptr_ok(S_new) || !ptr_ok(workspace))
     return TV_ERR_INVALID_ARG;
@@ -148,13 +164,14 @@ tv_status tv_get_status(void *workspace, tv_stream_t stream) {
   if (!ptr_ok(workspace)) return TV_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   int host[2] = {0, 0};
-  if (cudaMemcpyAsync(host, workspace, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    return TV_ERR_CUDA;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return TV_ERR_CUDA;
-  if (host[0] != TV_OK) {
-    if (cudaMemsetAsync(workspace, 0, sizeof(host), s) != cudaSuccess) return TV_ERR_CUDA;
-    if (cudaStreamSynchronize(s) != cudaSuccess) return TV_ERR_CUDA;
+  tv_status st = from_cuda(cudaMemcpyAsync(host, workspace, sizeof(host),
+                                           cudaMemcpyDeviceToHost, s));
+  if (st == TV_OK) st = from_cuda(cudaStreamSynchronize(s));
+  if (st == TV_OK && host[0] != TV_OK) {
+    st = from_cuda(cudaMemsetAsync(workspace, 0, sizeof(host), s));
+    if (st == TV_OK) st = from_cuda(cudaStreamSynchronize(s));
   }
+  if (st != TV_OK) return st;
   return static_cast<tv_status>(host[0]);
 }
 

@@ -13,10 +13,13 @@ The five named workloads mirror the shapes of the pages' setting:
 * ``config(2)``: gated delta rule, B=1, H=16, 16-node random tree of depth <= 6.
 * ``config(3)``: gated delta rule, B=32, H=32, 64-node trees of depth <= 8, branching 1..4.
 * ``config(4)``: gated delta rule, B=128, H=32, ragged trees of 8..48 nodes under a shared
-  batch-wide budget of 3072 nodes (the "batch-wide verification budget" of the Twig/Bole
-  abstract), depth <= 7.
+  batch-wide budget of 3072 nodes (the per-batch cap on verified nodes that the Twig/Bole
+  abstracts describe), depth <= 7.
 * ``config(5)``: gated delta rule, B=8, H=32, 256-node trees of depth <= 10, branching 1..8,
   near-1 decay.
+
+Outputs default to fp32 (``out_dtype``): rounding o to bf16 alone moves the largest
+outputs by up to 2^-9 of their size, which exceeds 2e-2 of the output RMS.
 
 Conventions: node indices inside a sequence are local (0..n_b-1) and topological
 (``parent[i] < i``); ``-1`` is the root state S_root.  The depth of a first-level draft node
@@ -233,7 +236,7 @@ def synthetic(parents: List[List[int]], H: int, dk: int, dv: int, *, seed: int,
         paths = [(_path_to(p, len(p) - 1) if len(p) else []) for p in parents]
     ap = _pad_paths(paths)
     return Workload(name=name, mode=mode, B=B, H=H, dk=dk, dv=dv, in_dtype=in_dtype,
-                    out_dtype=out_dtype or in_dtype, parent=parent, node_offsets=offsets,
+                    out_dtype=out_dtype or "f32", parent=parent, node_offsets=offsets,
                     q=q, k=k, v=v, log_a=log_a, b=b, S_root=S_root, accepted_path=ap,
                     max_nodes=max([1] + counts), max_path=ap.shape[1])
 
@@ -317,6 +320,6 @@ def config(idx: int, seed: int = 0) -> Workload:
     parent = np.concatenate([np.asarray(p, dtype=np.int32) for p in parents])
     ap = _pad_paths(paths)
     return Workload(name=f"config{idx}", mode="gdn", B=B, H=H, dk=dk, dv=dv, in_dtype="bf16",
-                    out_dtype="bf16", parent=parent, node_offsets=offsets, q=q, k=k, v=v,
+                    out_dtype="f32", parent=parent, node_offsets=offsets, q=q, k=k, v=v,
                     log_a=log_a, b=b, S_root=S_root, accepted_path=ap,
                     max_nodes=max(counts), max_path=ap.shape[1])
