@@ -5,10 +5,6 @@
 
 #include "tv_internal.cuh"
 
-#ifndef TV_HAVE_TC
-#define TV_HAVE_TC 0
-#endif
-
 namespace {
 
 using namespace tv;
@@ -38,8 +34,8 @@ tv_status check_problem(const tv_problem *p) {
 bool ptr_ok(const void *ptr) { return ptr && aligned16(ptr); }
 
 bool tc_supports(const tv_problem *p) {
-  return TV_HAVE_TC && p->in_dtype == TV_BF16 && p->dk == 128 && p->dv == 128 &&
-         p->max_nodes <= 64;
+  return p->in_dtype == TV_BF16 && p->dk == 128 && p->dv == 128 &&
+         p->max_nodes <= verify_tc_max_nodes();
 }
 
 thread_local cudaError_t g_last_cuda = cudaSuccess;

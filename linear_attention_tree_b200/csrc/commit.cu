@@ -5,22 +5,25 @@
 // (the Bole summary's worked example rebuilds S_c3 this way for scalar decay; with the
 // pseudo-values of the tree solve the same form holds for the gated delta rule).
 //
-// One CTA per (sequence, head).  The kernel is HBM bound (one read and one write of the
-// state), so the S_root loads are issued first, before anything that depends on the path;
-// the path is then checked by all threads at once, its rank-one factors are staged in
-// shared memory in chunks of kChunk entries, and S_new is streamed out with 128-bit stores.
+// One CTA per (sequence, head, slice of kRows state rows).  The kernel is HBM bound (one
+// read and one write of the state), so the S_root loads are issued first, before anything
+// that depends on the path; the path is then checked by all threads at once, its rank-one
+// factors are staged in shared memory in chunks of kChunk entries, and S_new is streamed
+// out with 128-bit stores.  Small CTAs keep many slices in flight per SM, which hides the
+// chain of dependent loads (offsets -> path -> parent, log_a -> u, k rows) of each slice.
 #include "tv_internal.cuh"
 
 namespace tv {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 128;
+constexpr int kRows = 32;                          // state rows (v) per CTA
 constexpr int kChunk = 16;
-constexpr int kMaxVec = 128 * 128 / 4 / kThreads;  // float4 slots per thread at dk=dv=128
+constexpr int kMaxVec = kRows * 128 / 4 / kThreads;  // float4 slots per thread at dk=128
 constexpr int kMaxPathWidth = 1024;
 
 struct CommitSmem {
-  float cu[kChunk][128];   // exp(c_m - c_j) u_{p_j}
+  float cu[kChunk][kRows]; // exp(c_m - c_j) u_{p_j}, this CTA's rows
   float kk[kChunk][128];   // k_{p_j}
   int prow[kMaxPathWidth]; // the accepted_path row
   float la[kMaxNodes];     // log_a of the path nodes
@@ -33,14 +36,17 @@ template <typename Tk>
 __global__ void __launch_bounds__(kThreads) commit_kernel(CommitArgs a) {
   __shared__ __align__(16) CommitSmem sm;
   const int tid = threadIdx.x;
-  const int s = blockIdx.x / a.H, h = blockIdx.x % a.H;
   const int H = a.H, dk = a.dk, dv = a.dv;
+  const int slices = (dv + kRows - 1) / kRows;
+  const int s = blockIdx.x / (H * slices), h = (blockIdx.x / slices) % H;
+  const int r0 = (blockIdx.x % slices) * kRows;           // first state row of the slice
+  const int rows = min(kRows, dv - r0);
   const Tk *k = static_cast<const Tk *>(a.k);
 
-  // 1. stream the state in (independent of everything else)
-  const size_t base = ((size_t)s * H + h) * dv * dk;
+  // 1. stream the state slice in (independent of everything else)
+  const size_t base = (((size_t)s * H + h) * dv + r0) * dk;
   const float4 *Sg = reinterpret_cast<const float4 *>(a.S_root + base);
-  const int nvec = dv * dk / 4;
+  const int nvec = rows * dk / 4;
   float4 acc[kMaxVec];
 #pragma unroll
   for (int r = 0; r < kMaxVec; ++r) {
@@ -52,7 +58,7 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(CommitArgs a) {
   const int lo = a.node_offsets[s], hi = a.node_offsets[s + 1];
   if (lo < 0 || hi < lo || hi > a.T || hi - lo > a.max_nodes ||
       (s == 0 && lo != 0) || (s == a.B - 1 && hi != a.T)) {
-    if (tid == 0) set_status(a.ws, TV_ERR_BAD_TREE, s);
+    if (tid == 0 && r0 == 0) set_status(a.ws, TV_ERR_BAD_TREE, s);
     return;
   }
   const int n_nodes = hi - lo;
@@ -78,7 +84,7 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(CommitArgs a) {
   }
   __syncthreads();
   if (sm.flag) {
-    if (tid == 0) set_status(a.ws, TV_ERR_BAD_PATH, s);
+    if (tid == 0 && r0 == 0) set_status(a.ws, TV_ERR_BAD_PATH, s);
     return;
   }
   if (tid == 0) {
@@ -103,7 +109,7 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(CommitArgs a) {
     for (int e = tid; e < cnt * 128; e += kThreads) {
       const int j = e / 128, x = e % 128;
       const size_t node = (size_t)(lo + sm.prow[j0 + j]) * H + h;
-      if (x < dv) sm.cu[j][x] = expf(cm - sm.c[j0 + j]) * a.U[node * dv + x];
+      if (x < rows) sm.cu[j][x] = expf(cm - sm.c[j0 + j]) * a.U[node * dv + r0 + x];
       if (x < dk) sm.kk[j][x] = to_f32(k[node * dk + x]);
     }
     __syncthreads();
@@ -138,10 +144,11 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(CommitArgs a) {
 int commit_max_path_width() { return kMaxPathWidth; }
 
 cudaError_t launch_commit(const CommitArgs &a, int in_dtype, cudaStream_t st) {
+  const int grid = a.B * a.H * ((a.dv + kRows - 1) / kRows);
   if (in_dtype == TV_F32)
-    commit_kernel<float><<<a.B * a.H, kThreads, 0, st>>>(a);
+    commit_kernel<float><<<grid, kThreads, 0, st>>>(a);
   else
-    commit_kernel<__nv_bfloat16><<<a.B * a.H, kThreads, 0, st>>>(a);
+    commit_kernel<__nv_bfloat16><<<grid, kThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -65,6 +65,7 @@ struct MetaArgs {
 // Launchers (host side); each returns cudaSuccess or the launch error.
 cudaError_t launch_verify_simt(const VerifyArgs &a, int mode, int in_dtype, int out_dtype,
                                cudaStream_t st);
+int verify_tc_max_nodes();
 cudaError_t launch_verify_tc(const VerifyArgs &a, int mode, int out_dtype, cudaStream_t st);
 int commit_max_path_width();
 cudaError_t launch_commit(const CommitArgs &a, int in_dtype, cudaStream_t st);

@@ -20,7 +20,7 @@ def _verify(w, d, ws, kernel="auto", **kw):
                          workspace=ws, kernel=kernel, **kw)
 
 
-@pytest.mark.parametrize("kernel", ["auto", "simt"])
+@pytest.mark.parametrize("kernel", ["tc", "simt"])
 @pytest.mark.parametrize("bad", ["self_parent", "forward_parent", "below_minus_one",
                                  "offsets_decreasing", "offsets_too_many"])
 def test_bad_tree(kernel, bad):
@@ -75,7 +75,7 @@ def test_bad_path(bad):
     assert_close(S_new[5, 3].cpu().numpy(), want, TOL["bf16"], "other sequence")
 
 
-@pytest.mark.parametrize("kernel", ["auto", "simt"])
+@pytest.mark.parametrize("kernel", ["tc", "simt"])
 def test_guard_regions_untouched(kernel):
     """Outputs carved out of larger NaN-filled buffers: nothing outside is written."""
     pars = [W.frontier_tree(50 + i, c, 8, 4)[0] for i, c in enumerate([63, 1, 64, 17])]

@@ -11,7 +11,7 @@ from tests._gpu_util import TOL, assert_close, run
 
 pytestmark = pytest.mark.gpu
 
-KERNELS = ["auto", "simt"]
+KERNELS = ["tc", "simt"]
 
 
 @pytest.mark.parametrize("kernel", KERNELS)

@@ -57,14 +57,24 @@ def test_config1_worked_example(kernel):
     _full_check(W.config(1), kernel)
 
 
-@pytest.mark.parametrize("kernel", ["auto", "simt"])
+@pytest.mark.parametrize("kernel", ["auto", "simt", "tc"])
 def test_config2(kernel):
     _full_check(W.config(2), kernel)
 
 
 @pytest.mark.parametrize("idx", [3, 4, 5])
 def test_full_size_sampled(idx):
+    """Default kernel choice, as the benchmark runs it (tensor cores up to 64 nodes)."""
     _sampled_check(W.config(idx))
+
+
+def test_tc_matches_simt_config3():
+    """The two kernels agree far inside the oracle bar (bf16 S_root products aside)."""
+    w = W.config(3)
+    a, _ = run(w, kernel="tc")
+    b, _ = run(w, kernel="simt")
+    for key in ("o", "U", "S_new"):
+        assert_close(a[key], b[key], 5e-3, key + " tc vs simt")
 
 
 @pytest.mark.parametrize("idx", [3, 4, 5])
@@ -85,8 +95,8 @@ def _ragged(seed, counts, max_depth=8, fmax=4):
     return pars
 
 
-@pytest.mark.parametrize("kernel", ["auto", "simt"])
-@pytest.mark.parametrize("counts", [[64, 37, 9], [1, 63, 64, 2], [5, 0, 17]])
+@pytest.mark.parametrize("kernel", ["tc", "simt"])
+@pytest.mark.parametrize("counts", [[64, 37, 9], [1, 63, 64, 2], [5, 0, 17], [64] * 5])
 def test_ragged_small_full(kernel, counts):
     """Several sequences, ragged node counts (incl. an empty tree), compared in full."""
     w = W.synthetic(_ragged(len(counts), counts), H=3, dk=128, dv=128,
@@ -103,7 +113,7 @@ def test_dims_f32(mode, dk, dv):
     _full_check(w, "simt")
 
 
-@pytest.mark.parametrize("kernel", ["auto", "simt"])
+@pytest.mark.parametrize("kernel", ["tc", "simt"])
 def test_scalar_bf16(kernel):
     pars = _ragged(5, [40, 64])
     w = W.synthetic(pars, H=2, dk=128, dv=128, seed=5, mode="scalar", log_a_mean=-3.0)
