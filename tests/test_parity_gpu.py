@@ -69,12 +69,17 @@ def test_full_size_sampled(idx):
 
 
 def test_tc_matches_simt_config3():
-    """The two kernels agree far inside the oracle bar (bf16 S_root products aside)."""
+    """The two kernels agree at half the oracle bar over the whole workload.
+
+    The tensor-core kernel rounds S_root to bf16 for the state products and rounds the
+    operands of its second (tf32) product to nearest; together that moves o by up to about
+    0.6% of its RMS, while the CUDA-core kernel stays at fp32 rounding.
+    """
     w = W.config(3)
     a, _ = run(w, kernel="tc")
     b, _ = run(w, kernel="simt")
     for key in ("o", "U", "S_new"):
-        assert_close(a[key], b[key], 5e-3, key + " tc vs simt")
+        assert_close(a[key], b[key], 1e-2, key + " tc vs simt")
 
 
 @pytest.mark.parametrize("idx", [3, 4, 5])
