@@ -2,26 +2,29 @@
 // per tree, gated delta rule or scalar decay.
 //
 // Notation for one (sequence, head) item: N <= 64 nodes in topological order, path(n) =
-// strict ancestors anc(n) plus n, cl_n = fp32 sum of log_a over path(n) (root first),
-// gamma_n = exp(cl_n), D[n][i] = exp(cl_n - cl_i).
+// strict ancestors anc(n) plus n (root first, indices increase along it), cl_n = fp32 sum
+// of log_a over path(n) (root first), gamma_n = exp(cl_n), D[n][i] = exp(cl_n - cl_i).
 //
-// MMA 1 (tcgen05 kind::f16, 128 x 192 x 128, bf16 in, fp32 accumulate in TMEM):
+// MMA (tcgen05 kind::f16, 128 x 192 x 128, bf16 in, fp32 accumulate in TMEM):
 //      [ Q ] . [ K ; S_root ]^T  ->  [ Q K^T | (S_root Q^T)^T ]   rows 0..63
 //      [ K ]                         [ K K^T | (S_root K^T)^T ]   rows 64..127
-// gives both path Gram blocks and both state products at once.  q, k, v arrive by TMA in
-// the 128-byte swizzled layout the MMA reads; S_root (fp32 in HBM) is converted to bf16 by
-// all threads straight into the same layout.
+// gives both path Gram blocks and both state products -- the only dense contraction of
+// the method.  q, k, v arrive by TMA in the 128-byte swizzled layout the MMA reads;
+// S_root (fp32 in HBM) is converted to bf16 by all threads straight into the same layout.
 //
 // The tree system (tree-structured WY form of the TreeWY abstract) is
 //      (I + L) U = R,  L[n][i] = b_n D[n][i] k_n.k_i (i in anc(n)),  R_n = b_n (v_n - gamma_n S_root k_n)
 // and the outputs (closed form of the Bole summary's worked example, "具体技术细节示例",
-// extended to the delta rule) are  O = diag(gamma) S_root Q^T + P U  with
+// extended to the delta rule) are  o_n = gamma_n S_root q_n + sum_i P[n][i] u_i  with
 // P[n][i] = D[n][i] q_n.k_i on path(n).  With T = (I + L)^-1 and W = P T:
-//      U = T R,      O = diag(gamma) S_root Q^T + W R .
-// Rows of T and W live on the node's own path and follow from L alone by a backward
-// recursion along that path (T (I + L) = I, W (I + L) = P): one thread per row, no
-// barriers.  MMA 2 (kind::tf32, 128 x 128 x 64, operands rounded to nearest tf32) forms
-// [ W ; T ] . R in TMEM.  Scalar decay is the special case L = 0 (T = I, W = P, U = R = V).
+//      u_n = sum_{i in path(n)} T[n][i] R_i,      o_n = gamma_n S_root q_n + sum_{i in path(n)} W[n][i] R_i .
+// The decays factor out of both rows: T[n][i] = D[n][i] tau_i, W[n][i] = D[n][i] omega_i,
+// where along path(n) = p_0 .. p_{d-1} = n (right-looking, deepest first)
+//      tau_{d-1} = 1,             tau_a   = - sum_{c > a} tau_c   b_{p_c} k_{p_c}.k_{p_a}
+//      omega_a = q_n.k_{p_a}                - sum_{c > a} omega_c b_{p_c} k_{p_c}.k_{p_a}
+// so each row is one thread's short register recursion, and the path sums are fp32 FMAs
+// with one warp per node row, written straight to HBM.  Scalar decay: tau = e_{d-1}
+// (u_n = v_n), omega_a = q_n.k_{p_a}.
 //
 // Scheduling: one persistent CTA per SM walks the items blockIdx.x, +gridDim.x, ...
 // While item i is in its epilogue, item i+1's S_root is already streaming into registers
@@ -41,30 +44,43 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kTile = 64;                  // nodes per tree handled by this kernel
-constexpr uint32_t kTmemCols = 512;        // accumulator 1: cols 0..191, accumulator 2: 256..383
-constexpr uint32_t kAcc2 = 256;
+constexpr int kRegDepth = 16;              // deeper paths take the shared-memory recursion
+constexpr uint32_t kTmemCols = 256;        // accumulator: columns 0..191
 constexpr uint32_t kSpinLimit = 1u << 22;  // polls before a wait is declared timed out
 
 // Dynamic shared memory, offsets from a 1024-byte aligned base.
-constexpr int kOpHalf = 256 * 128;         // one 64-wide K half of [Q ; K ; S_root]
-constexpr int kOffOp = 0;                  // MMA 1 operands, 64 KiB
+//   [0, 64K)      MMA operands: two 64-wide K halves of [Q ; K ; S_root] (256 rows x 128 B).
+//                 Once the MMA is done, the next item's q/k land in rows 0..127 of each
+//                 half while rows 128..255 (the S_root rows) hold the T and W rows:
+//                 T at [16K, 32K), W at [48K, 64K) (64 x 64 fp32 each).
+//   [64K, 96K)    two v tiles (bf16, TMA swizzled)
+//   [96K, 128K)   R tile, 64 x 128 fp32
+//   [128K, 160K)  gamma_n S_root q_n tile, 64 x 128 fp32
+//   [160K, 176K)  b_j k_j.k_i on paths, 64 x 64 fp32
+//   [176K, 192K)  q_n.k_i on paths, 64 x 64 fp32
+//   [192K, 196K)  root-first path of every node (bytes)
+constexpr int kOpHalf = 256 * 128;
+constexpr int kOffOp = 0;
+constexpr int kOffT = 16384;
+constexpr int kOffW = 49152;
 constexpr int kVHalf = kTile * 128;
-constexpr int kOffV = 65536;               // two v tiles (bf16, TMA swizzled), 2 x 16 KiB
-constexpr int kOffB2 = 98304;              // R^T, MMA 2 B operand (fp32); then the O tile
-constexpr int kOffA2 = 131072;             // [W ; T], MMA 2 A operand (fp32); then the U tile
-constexpr int kAtom2 = 16384;              // one 32-wide K atom of a 128-row fp32 operand
-constexpr int kOffL = 163840;              // L coefficients, 64 x 64 fp32
-constexpr int kOffMisc = kOffL + kTile * kTile * 4;
+constexpr int kOffV = 65536;
+constexpr int kOffR = 98304;
+constexpr int kOffSQ = 131072;
+constexpr int kOffLK = 163840;
+constexpr int kOffGQ = 180224;
+constexpr int kOffPath = 196608;
+constexpr int kOffMisc = kOffPath + kTile * kTile;
 
 struct Misc {
   unsigned long long bar_tma;
-  unsigned long long bar_mma1;
-  unsigned long long bar_mma2;
+  unsigned long long bar_mma;
   unsigned long long anc[kTile];   // strict-ancestor bitmask
   uint32_t tmem_base;
   int timeout;
-  int outstanding[3];              // an issued TMA / MMA 1 / MMA 2 whose barrier was not waited
+  int outstanding[2];              // an issued TMA / MMA whose barrier was not waited
   int par[kTile];
+  int dep[kTile];
   float la[kTile];
   float bb[kTile];
   float cl[kTile];
@@ -72,28 +88,18 @@ struct Misc {
 constexpr int kSmemBytes = kOffMisc + (int)sizeof(Misc) + 1024;
 
 // fp32 [64][128] tile in four 32-column slabs of 128-byte rows with 16-byte chunks
-// XOR-swizzled by row: row-per-thread and column-per-thread accesses are conflict-free.
+// XOR-swizzled by row: row-per-thread and row-per-warp accesses are conflict-free.
 __device__ __forceinline__ int tile_off(int n, int v) {
   return ((v >> 5) << 13) + (n << 7) + ((((v >> 2) & 7) ^ (n & 7)) << 4) + ((v & 3) << 2);
 }
-// fp32 element (row, k) of a 128-row, K = 64 K-major operand with 128-byte swizzle.
-__device__ __forceinline__ int op2_off(int row, int k) {
-  return ((k >> 5) * kAtom2) + (row << 7) + ((((k >> 2) & 7) ^ (row & 7)) << 4) + ((k & 3) << 2);
-}
-// [64][64] fp32 coefficients, column XOR-swizzled by row.
-__device__ __forceinline__ int coef_off(int n, int i) { return (n << 6) + (i ^ (n & 31)); }
+// [64][64] fp32 matrix, column XOR-swizzled by row.
+__device__ __forceinline__ int coef_off(int n, int i) { return ((n << 6) + (i ^ (n & 31))) << 2; }
 
 __device__ __forceinline__ float lds(const unsigned char *p, int off) {
   return *reinterpret_cast<const float *>(p + off);
 }
 __device__ __forceinline__ void sts(unsigned char *p, int off, float x) {
   *reinterpret_cast<float *>(p + off) = x;
-}
-// fp32 -> nearest tf32 (ties away), kept in an fp32 container with the low 13 bits clear.
-__device__ __forceinline__ float tf32_rn(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return __uint_as_float(r);
 }
 
 struct Item {
@@ -153,6 +159,52 @@ __device__ __forceinline__ void load_meta(const VerifyArgs &a, const Item &x, in
   }
 }
 
+// Row recursion of node m (d = depth, path bytes `pth`): x_a for a < d with
+//   x_a = x0_a - sum_{c > a} x_c b_{p_c} k_{p_c}.k_{p_a}   (x0 = e_{d-1} for T, q_m.k for W)
+// then stores D[m][p_a] x_a into `dst` row m.  Register version for d <= kRegDepth.
+template <bool kW>
+__device__ __forceinline__ void row_recursion(unsigned char *sm, const uint8_t *pth, int m, int d,
+                                              const Misc &ms, int dst) {
+  const float clm = ms.cl[m];
+  if (d <= kRegDepth) {
+    int p[kRegDepth];
+    float x[kRegDepth];
+#pragma unroll
+    for (int a = 0; a < kRegDepth; ++a) {
+      p[a] = a < d ? pth[a] : 0;
+      x[a] = kW ? (a < d ? lds(sm, kOffGQ + coef_off(m, p[a])) : 0.f) : (a == d - 1 ? 1.f : 0.f);
+    }
+#pragma unroll
+    for (int c = kRegDepth - 1; c >= 1; --c) {
+      if (c < d) {
+        const float xc = x[c];
+#pragma unroll
+        for (int a = 0; a < c; ++a)
+          x[a] = fmaf(-xc, lds(sm, kOffLK + coef_off(p[c], p[a])), x[a]);
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < kRegDepth; ++a)
+      if (a < d) sts(sm, dst + coef_off(m, p[a]), x[a] * expf(clm - ms.cl[p[a]]));
+  } else {
+    // deep path: the row itself is the working storage (other rows are only read from LK)
+    for (int a = 0; a < d; ++a)
+      sts(sm, dst + coef_off(m, pth[a]),
+          kW ? lds(sm, kOffGQ + coef_off(m, pth[a])) : (a == d - 1 ? 1.f : 0.f));
+    for (int c = d - 1; c >= 1; --c) {
+      const float xc = lds(sm, dst + coef_off(m, pth[c]));
+      for (int a = 0; a < c; ++a) {
+        const int o = dst + coef_off(m, pth[a]);
+        sts(sm, o, fmaf(-xc, lds(sm, kOffLK + coef_off(pth[c], pth[a])), lds(sm, o)));
+      }
+    }
+    for (int a = 0; a < d; ++a) {
+      const int o = dst + coef_off(m, pth[a]);
+      sts(sm, o, lds(sm, o) * expf(clm - ms.cl[pth[a]]));
+    }
+  }
+}
+
 template <bool kGdn, typename Tout>
 __global__ void __launch_bounds__(kThreads, 1)
     verify_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -162,6 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char *sm = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
   Misc &ms = *reinterpret_cast<Misc *>(sm + kOffMisc);
+  uint8_t *paths = reinterpret_cast<uint8_t *>(sm + kOffPath);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int num_items = a.B * a.H;
   int it = blockIdx.x;
@@ -169,20 +222,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const uint32_t sbase = ptx::smem_addr(sm);
   const uint32_t bar_tma = ptx::smem_addr(&ms.bar_tma);
-  const uint32_t bar_mma1 = ptx::smem_addr(&ms.bar_mma1);
-  const uint32_t bar_mma2 = ptx::smem_addr(&ms.bar_mma2);
+  const uint32_t bar_mma = ptx::smem_addr(&ms.bar_mma);
 
   // ---- prologue: barriers, tensor memory, first item's loads --------------------------
   Item cur = load_item(a, it);
   if (tid == 0) {
     ptx::mbar_init(bar_tma, 1);
-    ptx::mbar_init(bar_mma1, 1);
-    ptx::mbar_init(bar_mma2, 1);
+    ptx::mbar_init(bar_mma, 1);
     ptx::fence_mbar_init();
     ms.timeout = 0;
     ms.outstanding[0] = 1;
     ms.outstanding[1] = 0;
-    ms.outstanding[2] = 0;
     ptx::prefetch_tmap(&tm_q);
     ptx::prefetch_tmap(&tm_k);
     ptx::prefetch_tmap(&tm_v);
@@ -208,13 +258,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n = is_q ? row : row - kTile;          // node of this thread's accumulator row
   const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
 
-  uint32_t ph_tma = 0, ph_m1 = 0, ph_m2 = 0;
+  uint32_t ph_tma = 0, ph_mma = 0;
   for (int local = 0; it < num_items; ++local, it += gridDim.x) {
     const int buf = local & 1;
     const int nxt = it + gridDim.x;
     const bool has_next = nxt < num_items;
-    Item nx;
-    if (has_next) nx = load_item(a, nxt);
     const int n_nodes = cur.n;
 
     // ---- 1. state -> bf16 operand rows 128..255; tree metadata -> shared --------------
@@ -247,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool bad_tree = __syncthreads_or(bad) != 0 || !cur.ok;
     const bool run = !bad_tree && n_nodes > 0;
 
-    // ---- 2. MMA 1 (one thread); metadata walk; next item's state and metadata loads ---
+    // ---- 2. MMA (one thread); paths and decays; the next item's loads -----------------
     if (tid == kThreads - 1) {
       const bool landed = ptx::mbar_wait_bounded(bar_tma, ph_tma, kSpinLimit);
       if (landed) ms.outstanding[0] = 0;
@@ -262,27 +310,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ptx::smem_desc_sw128(base + kTile * 128, 1024), idesc, kk > 0 ? 1u : 0u);
         }
         ms.outstanding[1] = 1;
-        ptx::mma_commit(bar_mma1);
+        ptx::mma_commit(bar_mma);
       }
     }
     ph_tma ^= 1u;
+    Item nx;
+    if (has_next) nx = load_item(a, nxt);
+    if (has_next) load_state(a, nx, tid, sreg);
     if (tid < kTile) {
-      // strict ancestors by walking up; cl summed root first (ancestor indices increase
-      // with depth, so ascending bit order is path order)
+      // walk up: ancestor bits, depth, root-first path bytes; cl summed root first
       unsigned long long bits = 0ull;
+      int d = 0;
       float cl = 0.f;
       if (run && tid < n_nodes) {
-        for (int x = ms.par[tid]; x >= 0; x = ms.par[x]) bits |= 1ull << x;
-        for (unsigned long long b = bits; b; b &= b - 1) cl += ms.la[__ffsll((long long)b) - 1];
-        cl += ms.la[tid];
+        d = 1;
+        for (int x = ms.par[tid]; x >= 0; x = ms.par[x]) {
+          bits |= 1ull << x;
+          ++d;
+        }
+        uint8_t *pth = paths + tid * kTile;
+        pth[d - 1] = (uint8_t)tid;
+        int pos = d - 2;
+        for (int x = ms.par[tid]; x >= 0; x = ms.par[x]) pth[pos--] = (uint8_t)x;
+        for (int t = 0; t < d; ++t) cl += ms.la[pth[t]];
       }
       ms.anc[tid] = bits;
+      ms.dep[tid] = d;
       ms.cl[tid] = cl;
     }
-    if (has_next) {
-      load_state(a, nx, tid, sreg);
-      load_meta<kGdn>(a, nx, tid, p_reg, la_reg, bb_reg);
-    }
+    if (has_next) load_meta<kGdn>(a, nx, tid, p_reg, la_reg, bb_reg);
     __syncthreads();
     if (ms.timeout) break;
     if (bad_tree && tid == 0) set_status(a.ws, TV_ERR_BAD_TREE, cur.s);
@@ -290,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- 3. operands consumed: prefetch the next item's q / k / v ---------------------
     if (tid == 0) {
       if (run) {
-        if (ptx::mbar_wait_bounded(bar_mma1, ph_m1, kSpinLimit)) ms.outstanding[1] = 0;
+        if (ptx::mbar_wait_bounded(bar_mma, ph_mma, kSpinLimit)) ms.outstanding[1] = 0;
         else ms.timeout = 1;
       }
       if (has_next && !ms.timeout) {
@@ -298,55 +354,56 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_tma(nx, buf ^ 1, sbase, bar_tma, &tm_q, &tm_k, &tm_v);
       }
     }
-    if (run) ph_m1 ^= 1u;
+    if (run) ph_mma ^= 1u;
     __syncthreads();
     if (ms.timeout) break;
 
     if (run) {
       ptx::tc_fence_after();
       const bool live = n < n_nodes;
-      const float cln = ms.cl[n];
-      const float gam = expf(cln);
+      const float gam = expf(ms.cl[n]);
       const unsigned long long ancn = ms.anc[n];
       const unsigned long long pathn = live ? (ancn | (1ull << n)) : 0ull;
       const unsigned char *vt = sm + kOffV + buf * 2 * kVHalf;
 
-      // ---- 4. accumulator 1 -> R^T (B2), raw Gram on paths (L, and P in A2's W rows) --
-      if (!is_q) {
+      // ---- 4. accumulator -> R and gamma S_root q tiles, path Gram entries -------------
+      // warp w reads TMEM lanes 32*(w%4)..; warps 0-3 take value columns 0..63 and Gram
+      // columns 0..31, warps 4-7 value columns 64..127 and Gram columns 32..63.
+      {
         const float bn = ms.bb[n];
+        unsigned char *tile = sm + (is_q ? kOffSQ : kOffR);
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           float x[16];
           const int v0 = set * 64 + c * 16;
           ptx::tmem_ld16(trow + 64 + v0, x);
-          const int half = v0 >> 6, ch = (v0 & 63) >> 3;
-          const uint4 w0 = *reinterpret_cast<const uint4 *>(
-              vt + half * kVHalf + (n << 7) + ((ch ^ (n & 7)) << 4));
-          const uint4 w1 = *reinterpret_cast<const uint4 *>(
-              vt + half * kVHalf + (n << 7) + (((ch + 1) ^ (n & 7)) << 4));
-          const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float vn = __uint_as_float(((wv[j >> 1] >> ((j & 1) * 16)) & 0xFFFFu) << 16);
-            const float rr = kGdn ? bn * (vn - gam * x[j]) : vn;
-            sts(sm, kOffB2 + op2_off(v0 + j, n), live ? tf32_rn(rr) : 0.f);
-          }
-        }
-        if (kGdn) {
-          float *L = reinterpret_cast<float *>(sm + kOffL);
-#pragma unroll 1
-          for (int c = 0; c < 2; ++c) {
-            float g[16];
-            const int i0 = set * 32 + c * 16;
-            ptx::tmem_ld16(trow + i0, g);
+          if (is_q) {
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              if ((ancn >> (i0 + j)) & 1ull) L[coef_off(n, i0 + j)] = g[j];
+            for (int j = 0; j < 16; ++j) x[j] *= gam;
+          } else {
+            const int half = v0 >> 6, ch = (v0 & 63) >> 3;
+            const uint4 w0 = *reinterpret_cast<const uint4 *>(
+                vt + half * kVHalf + (n << 7) + ((ch ^ (n & 7)) << 4));
+            const uint4 w1 = *reinterpret_cast<const uint4 *>(
+                vt + half * kVHalf + (n << 7) + (((ch + 1) ^ (n & 7)) << 4));
+            const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float vn = __uint_as_float(((wv[j >> 1] >> ((j & 1) * 16)) & 0xFFFFu) << 16);
+              x[j] = live ? (kGdn ? bn * (vn - gam * x[j]) : vn) : 0.f;
+            }
           }
+#pragma unroll
+          for (int j = 0; j < 16; j += 4)
+            *reinterpret_cast<float4 *>(tile + tile_off(n, v0 + j)) =
+                make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
         }
-      } else {
+        // Gram on paths: K rows -> b_n k_n.k_i (i in anc(n)), Q rows -> q_n.k_i (i in path(n))
+        const int gbase = is_q ? kOffGQ : kOffLK;
+        const unsigned long long sel = is_q ? pathn : (live ? ancn : 0ull);
+        const float scale = is_q ? 1.f : bn;
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
           float g[16];
@@ -355,141 +412,72 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            sts(sm, kOffA2 + op2_off(n, i0 + j), ((pathn >> (i0 + j)) & 1ull) ? g[j] : 0.f);
+            if ((sel >> (i0 + j)) & 1ull) sts(sm, gbase + coef_off(n, i0 + j), scale * g[j]);
         }
       }
       ptx::tc_fence_before();
       __syncthreads();
 
-      // ---- 5. decays on L (one thread per node): L[m][i] = b_m D[m][i] k_m.k_i ---------
-      float *L = reinterpret_cast<float *>(sm + kOffL);
-      if (kGdn && tid < n_nodes) {
-        const int m = tid;
-        const float clm = ms.cl[m], bm = ms.bb[m];
-        for (unsigned long long bi = ms.anc[m]; bi; bi &= bi - 1) {
-          const int i = __ffsll((long long)bi) - 1;
-          L[coef_off(m, i)] *= bm * expf(clm - ms.cl[i]);
-        }
-      }
-      __syncthreads();
-
-      // ---- 6. rows of W (tid < 64) and T (tid 64..127) by backward recursion ------------
-      //   W[m][i] = P[m][i] - sum_{j in path(m), j > i} W[m][j] L[j][i]
-      //   T[m][i] =  I[m][i] - sum_{j in path(m), j > i} T[m][j] L[j][i]
-      // for i in anc(m), deepest first (ancestor indices increase with depth).
+      // ---- 5. T rows (threads 0..63) and W rows (threads 64..127) ----------------------
       if (tid < 2 * kTile) {
-        const bool do_t = tid >= kTile;
-        const int m = do_t ? tid - kTile : tid;
-        const int r2 = do_t ? kTile + m : m;
-        if (do_t) {
-          const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int c = 0; c < 16; ++c)
-            *reinterpret_cast<float4 *>(sm + kOffA2 + op2_off(r2, c * 4)) = z;
-          if (m < n_nodes) sts(sm, kOffA2 + op2_off(r2, m), 1.f);
-        }
+        const int m = tid & (kTile - 1);
         if (m < n_nodes) {
-          const unsigned long long am = ms.anc[m];
-          const float clm = ms.cl[m];
-          if (!do_t)   // P[m][i] = D[m][i] q_m.k_i
-            for (unsigned long long bi = am; bi; bi &= bi - 1) {
-              const int i = __ffsll((long long)bi) - 1;
-              const int o = kOffA2 + op2_off(r2, i);
-              sts(sm, o, lds(sm, o) * expf(clm - ms.cl[i]));
+          const int d = ms.dep[m];
+          const uint8_t *pth = paths + m * kTile;
+          if (tid < kTile) {
+            if (kGdn) {
+              row_recursion<false>(sm, pth, m, d, ms, kOffT);
+            } else {
+              for (int a2 = 0; a2 < d; ++a2) sts(sm, kOffT + coef_off(m, pth[a2]), a2 == d - 1 ? 1.f : 0.f);
             }
-          if (kGdn) {
-            const float selfc = lds(sm, kOffA2 + op2_off(r2, m));
-            for (unsigned long long bi = am; bi;) {
-              const int i = 63 - __clzll((long long)bi);
-              bi ^= 1ull << i;
-              float acc = do_t ? 0.f : lds(sm, kOffA2 + op2_off(r2, i));
-              acc = fmaf(-selfc, L[coef_off(m, i)], acc);
-              for (unsigned long long bj = am & ~((2ull << i) - 1ull); bj; bj &= bj - 1) {
-                const int j = __ffsll((long long)bj) - 1;
-                acc = fmaf(-lds(sm, kOffA2 + op2_off(r2, j)), L[coef_off(j, i)], acc);
+          } else {
+            if (kGdn) {
+              row_recursion<true>(sm, pth, m, d, ms, kOffW);
+            } else {
+              const float clm = ms.cl[m];
+              for (int a2 = 0; a2 < d; ++a2) {
+                const int i = pth[a2];
+                sts(sm, kOffW + coef_off(m, i), lds(sm, kOffGQ + coef_off(m, i)) * expf(clm - ms.cl[i]));
               }
-              sts(sm, kOffA2 + op2_off(r2, i), acc);
             }
           }
-          // operands of the tf32 MMA, rounded to nearest
-          for (unsigned long long bi = am | (1ull << m); bi; bi &= bi - 1) {
-            const int o = kOffA2 + op2_off(r2, __ffsll((long long)bi) - 1);
-            sts(sm, o, tf32_rn(lds(sm, o)));
-          }
         }
       }
-      ptx::fence_proxy_async_smem();
-      ptx::tc_fence_before();
       __syncthreads();
 
-      // ---- 7. MMA 2: [W ; T] . R  (tf32, 128 x 128 x 64) -> TMEM columns 256..383 ------
-      if (tid == kThreads - 1) {
-        ptx::tc_fence_after();
-        constexpr uint32_t idesc = ptx::idesc_tf32_f32(128, 128);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t koff = (kk >> 2) * kAtom2 + (kk & 3) * 32;
-          ptx::mma_tf32(tmem + kAcc2, ptx::smem_desc_sw128(sbase + kOffA2 + koff, 1024),
-                        ptx::smem_desc_sw128(sbase + kOffB2 + koff, 1024), idesc,
-                        kk > 0 ? 1u : 0u);
-        }
-        ms.outstanding[2] = 1;
-        ptx::mma_commit(bar_mma2);
-      }
-      __syncthreads();
-      if (tid == 0) {
-        if (ptx::mbar_wait_bounded(bar_mma2, ph_m2, kSpinLimit)) ms.outstanding[2] = 0;
-        else ms.timeout = 1;
-      }
-      ph_m2 ^= 1u;
-      __syncthreads();
-      if (ms.timeout) break;
-      ptx::tc_fence_after();
-
-      // ---- 8. epilogue: o = gamma S_root q + (W R), u = (T R) -> O / U tiles ------------
-      unsigned char *tile = sm + (is_q ? kOffB2 : kOffA2);
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        const int v0 = set * 64 + c * 16;
-        float y[16];
-        ptx::tmem_ld16(trow + kAcc2 + v0, y);
-        if (is_q) {
-          float x[16];
-          ptx::tmem_ld16(trow + 64 + v0, x);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) y[j] = fmaf(gam, x[j], y[j]);
-        } else {
-          ptx::tmem_wait_ld();
-        }
-#pragma unroll
-        for (int j = 0; j < 16; j += 4)
-          *reinterpret_cast<float4 *>(tile + tile_off(n, v0 + j)) =
-              make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
-      }
-      ptx::tc_fence_before();
-      __syncthreads();
-
-      // ---- 9. coalesced rows out: a warp writes one 512-byte row per instruction ---------
+      // ---- 6. path sums, one warp per node row, straight to HBM -----------------------
+      //   u_m = sum_{i in path(m)} T[m][i] R_i,   o_m = gamma_m S_root q_m + sum_i W[m][i] R_i
       Tout *out = static_cast<Tout *>(a.out);
       const int v4 = lane * 4;
-      for (int r = warp; r < 2 * n_nodes; r += kThreads / 32) {
-        const bool is_u = r >= n_nodes;
-        const int m = is_u ? r - n_nodes : r;
-        const float4 x = *reinterpret_cast<const float4 *>(sm + (is_u ? kOffA2 : kOffB2) + tile_off(m, v4));
+      for (int m = warp; m < n_nodes; m += kThreads / 32) {
+        const int d = ms.dep[m];
+        const uint8_t *pth = paths + m * kTile;
+        float4 o4 = *reinterpret_cast<const float4 *>(sm + kOffSQ + tile_off(m, v4));
+        float4 u4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int a2 = 0; a2 < d; ++a2) {
+          const int i = pth[a2];
+          const float ct = lds(sm, kOffT + coef_off(m, i));
+          const float cw = lds(sm, kOffW + coef_off(m, i));
+          const float4 r4 = *reinterpret_cast<const float4 *>(sm + kOffR + tile_off(i, v4));
+          u4.x = fmaf(ct, r4.x, u4.x); u4.y = fmaf(ct, r4.y, u4.y);
+          u4.z = fmaf(ct, r4.z, u4.z); u4.w = fmaf(ct, r4.w, u4.w);
+          o4.x = fmaf(cw, r4.x, o4.x); o4.y = fmaf(cw, r4.y, o4.y);
+          o4.z = fmaf(cw, r4.z, o4.z); o4.w = fmaf(cw, r4.w, o4.w);
+        }
         const size_t g = ((size_t)(cur.lo + m) * a.H + cur.h) * 128 + v4;
-        if (is_u) {
-          __stcs(reinterpret_cast<float4 *>(a.U + g), x);
-        } else if (sizeof(Tout) == 4) {
-          __stcs(reinterpret_cast<float4 *>(reinterpret_cast<float *>(out) + g), x);
+        __stcs(reinterpret_cast<float4 *>(a.U + g), u4);
+        if (sizeof(Tout) == 4) {
+          __stcs(reinterpret_cast<float4 *>(reinterpret_cast<float *>(out) + g), o4);
         } else {
-          __nv_bfloat162 l2 = __floats2bfloat162_rn(x.x, x.y), h2 = __floats2bfloat162_rn(x.z, x.w);
+          __nv_bfloat162 l2 = __floats2bfloat162_rn(o4.x, o4.y), h2 = __floats2bfloat162_rn(o4.z, o4.w);
           uint2 pk;
           pk.x = *reinterpret_cast<uint32_t *>(&l2);
           pk.y = *reinterpret_cast<uint32_t *>(&h2);
           *reinterpret_cast<uint2 *>(reinterpret_cast<__nv_bfloat16 *>(out) + g) = pk;
         }
       }
+      // the next item's state conversion overwrites the T / W rows read above
+      __syncthreads();
     }
     if (has_next) cur = nx;
   }
@@ -498,8 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (ms.timeout && tid == 0) {
     set_status(a.ws, TV_ERR_TIMEOUT, blockIdx.x);
     if (ms.outstanding[0]) ptx::mbar_wait_bounded(bar_tma, ph_tma, kSpinLimit);
-    if (ms.outstanding[1]) ptx::mbar_wait_bounded(bar_mma1, ph_m1, kSpinLimit);
-    if (ms.outstanding[2]) ptx::mbar_wait_bounded(bar_mma2, ph_m2, kSpinLimit);
+    if (ms.outstanding[1]) ptx::mbar_wait_bounded(bar_mma, ph_mma, kSpinLimit);
   }
   ptx::tc_fence_before();
   __syncthreads();
