@@ -160,6 +160,28 @@ TV_API tv_status tv_tree_meta(const tv_problem *p, const int32_t *parent,
                        uint64_t *anc, float *cumlog, void *workspace,
                        size_t workspace_bytes, tv_stream_t stream);
 
+/* tv_tree_verify for callers that cannot allocate device memory when they verify: code
+ * running inside an allocator or memory-pool callback, serving loops that forbid
+ * allocation after start-up, hosts that hand over only buffers they own.  (The pages
+ * describe no such interface; this is a deployment convenience with no counterpart there.)
+ * Same arguments, layouts and results as tv_tree_verify, minus the workspace: the device
+ * scratch (the status word) is a fixed 4096-byte array inside this library's device image,
+ * held by every GPU that loads the library until the process exits.  Nothing is
+ * allocated and no allocating routine is called.
+ *   scratch_out  (host, may be NULL) receives the device address of that array, which can
+ *                be passed to tv_get_status to read and clear device-side errors.
+ * Problems whose tv_workspace_size exceeds 4096 bytes return TV_ERR_UNSUPPORTED.
+ * The first call on each device (with that device current) looks up the array's device
+ * address and zeroes it; make that first call before any stream capture.  All calls on a
+ * device share the one array, which keeps the last call's contents (a recorded error stays
+ * until tv_get_status clears it), so calls that overlap on the GPU, from different streams
+ * or threads, race on it. */
+TV_API tv_status tv_tree_verify_noalloc(const tv_problem *p, const void *q, const void *k,
+                                        const void *v, const float *log_a, const float *b,
+                                        const int32_t *parent, const int32_t *node_offsets,
+                                        const float *S_root, void *out, float *U,
+                                        void **scratch_out, tv_stream_t stream);
+
 /* Synchronise `stream`, return the first device-side error recorded in `workspace` since
  * the last call (TV_OK if none) and clear it.  Not for the hot path. */
 TV_API tv_status tv_get_status(void *workspace, tv_stream_t stream);
