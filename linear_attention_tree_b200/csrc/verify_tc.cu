@@ -78,6 +78,10 @@ struct Misc {
   unsigned long long anc[kTile];   // strict-ancestor bitmask
   uint32_t tmem_base;
   int flag;                        // 0, or a tv_status to record for this item
+  int maxdep;
+  // trees no deeper than kRegDepth keep the path Gram entries by path position:
+  float lpos[kTile][kRegDepth];    // b_j k_j.k_{a-th ancestor of j}
+  float gpos[kTile][kRegDepth];    // q_n.k_{a-th node of path(n)}
   int par[kTile];
   int dep[kTile];
   float la[kTile];
@@ -114,8 +118,9 @@ __device__ __forceinline__ float tf32_rn(float x) {
 // Row m of [W ; T] (A2 row `r2`): x_a for path positions a < d,
 //   x_a = x0_a - sum_{c > a} x_c lk[p_c][p_a]   (x0 = e_{d-1}: T row; x0 = gq row: W row)
 // (no recursion for scalar decay, where L = 0), times D[m][p_a], rounded to tf32 and
-// stored at column p_a.  Paths deeper than kRegDepth run in the A2 row itself, out of
-// line so that the register version stays small in the instruction cache.
+// stored at column p_a.  Trees deeper than kRegDepth run this in the A2 row itself on
+// dense Gram matrices, out of line so that the register version below (compact,
+// position-indexed Gram entries) stays small in the instruction cache.
 template <bool kW, bool kGdn>
 __device__ __noinline__ void row_coefficients_deep(unsigned char *sm, const uint8_t *paths,
                                                    const Misc &ms, int m, int d, int r2) {
@@ -144,24 +149,20 @@ __device__ __noinline__ void row_coefficients_deep(unsigned char *sm, const uint
 template <bool kW, bool kGdn>
 __device__ __forceinline__ void row_coefficients(unsigned char *sm, const uint8_t *paths,
                                                  const Misc &ms, int m, int d, int r2) {
-  if (d > kRegDepth) {
-    row_coefficients_deep<kW, kGdn>(sm, paths, ms, m, d, r2);
-    return;
-  }
   const float clm = ms.cl[m];
   int p[kRegDepth];
   float x[kRegDepth];
 #pragma unroll
   for (int a = 0; a < kRegDepth; ++a) {
     p[a] = a < d ? paths[a * kTile + m] : m;
-    x[a] = kW ? (a < d ? lds(sm, kOffGQ + coef_off(m, p[a])) : 0.f) : (a == d - 1 ? 1.f : 0.f);
+    x[a] = kW ? (a < d ? ms.gpos[m][a] : 0.f) : (a == d - 1 ? 1.f : 0.f);
   }
 #pragma unroll
   for (int c = kRegDepth - 1; c >= 1; --c) {
     if (kGdn && c < d) {
       const float xc = x[c];
 #pragma unroll
-      for (int a = 0; a < c; ++a) x[a] = fmaf(-xc, lds(sm, kOffLK + coef_off(p[c], p[a])), x[a]);
+      for (int a = 0; a < c; ++a) x[a] = fmaf(-xc, ms.lpos[p[c]][a], x[a]);
     }
   }
 #pragma unroll
@@ -182,7 +183,8 @@ template <bool kGdn, typename Tout>
 __global__ void __launch_bounds__(kThreads, 2)
     verify_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, VerifyArgs a) {
+                     const __grid_constant__ CUtensorMap tm_v, VerifyArgs a,
+                     int prefetch_stride) {
   extern __shared__ unsigned char smem_dyn[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
@@ -213,6 +215,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     ptx::mbar_init(bar_mma2, 1);
     ptx::fence_mbar_init();
     ms.flag = 0;
+    ms.maxdep = 0;
     ptx::prefetch_tmap(&tm_q);
     ptx::prefetch_tmap(&tm_k);
     ptx::prefetch_tmap(&tm_v);
@@ -290,6 +293,21 @@ __global__ void __launch_bounds__(kThreads, 2)
       ptx::mma_commit(bar_mma1);
     }
   }
+  if (tid == kThreads - 32) {
+    // L2 prefetch for the CTA one resident wave ahead: its S_root block and q / k / v tiles
+    const int nxt = blockIdx.x + prefetch_stride;
+    if (nxt < a.B * H) {
+      const int s2 = nxt / H, h2 = nxt % H;
+      ptx::prefetch_l2(a.S_root + (size_t)nxt * 128 * 128, 128 * 128 * 4);
+      const int lo2 = a.node_offsets[s2];
+      if (lo2 >= 0 && lo2 < a.T)
+        for (int half = 0; half < 2; ++half) {
+          ptx::prefetch_tile_l2(&tm_q, half * 64, h2, lo2);
+          ptx::prefetch_tile_l2(&tm_k, half * 64, h2, lo2);
+          ptx::prefetch_tile_l2(&tm_v, half * 64, h2, lo2);
+        }
+    }
+  }
   if (tid < kTile) {
     // ancestors in ascending index order are the root-first path; cl summed in that order
     unsigned long long bits = 0ull;
@@ -310,6 +328,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     ms.anc[tid] = bits;
     ms.dep[tid] = d;
     ms.cl[tid] = cl;
+    atomicMax(&ms.maxdep, d);
   }
   __syncthreads();
   if (bad_tree || ms.flag != 0) {
@@ -331,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     return;
   }
   ptx::tc_fence_after();
+  const bool fast = ms.maxdep <= kRegDepth;   // compact Gram entries, register recursion
 
   // ---- 3. accumulator 1 -> R (k lanes), gamma S_root q in place (q lanes), Gram ---------
   // warp w owns TMEM lanes 32*(w%4)..; warps 0-3 take value columns 0..63 and Gram
@@ -379,17 +399,29 @@ __global__ void __launch_bounds__(kThreads, 2)
         ptx::tmem_st16(trow + 64 + v0, z);
       }
     }
-    if (!is_q && kGdn) {   // b_n k_n.k_i on anc(n)
-      const unsigned long long sel = live ? ancn : 0ull;
+    // Gram entries: k lanes b_n k_n.k_i on anc(n) (gated delta only); q lanes (compact
+    // form only) q_n.k_i on path(n).  Position of node i on a path = ancestors below i.
+    if (is_q ? fast : kGdn) {
+      const unsigned long long sel = !live ? 0ull : (is_q ? (ancn | (1ull << n)) : ancn);
+      const float scale = is_q ? 1.f : bn;
+      float *posrow = is_q ? &ms.gpos[n][0] : &ms.lpos[n][0];
 #pragma unroll 1
       for (int c = 0; c < 2; ++c) {
         float g[16];
         const int i0 = set * 32 + c * 16;
         ptx::tmem_ld16(trow + i0, g);
+        const unsigned bits = (unsigned)(sel >> i0) & 0xFFFFu;
+        int pos = __popcll(sel & ((1ull << i0) - 1ull));   // path position of column i0
         ptx::tmem_wait_ld();
+        if (!fast) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if ((sel >> (i0 + j)) & 1ull) sts(sm, kOffLK + coef_off(n, i0 + j), bn * g[j]);
+          for (int j = 0; j < 16; ++j)
+            if ((bits >> j) & 1u) sts(sm, kOffLK + coef_off(n, i0 + j), scale * g[j]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if ((bits >> j) & 1u) posrow[pos++] = scale * g[j];
+        }
       }
     }
     // [W ; T] starts as zeros
@@ -401,7 +433,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   ptx::tmem_wait_st();
   ptx::tc_fence_before();
   __syncthreads();
-  if (is_q) {   // q_n.k_i on path(n), into the now free v tile
+  if (!fast) {
+  if (is_q) {   // dense q_n.k_i on path(n), into the now free v tile
     ptx::tc_fence_after();
     const unsigned long long sel = live ? (ancn | (1ull << n)) : 0ull;
 #pragma unroll 1
@@ -416,12 +449,18 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
   __syncthreads();
+  }
 
   // ---- 4. rows of W (warps 0-1) and T (warps 2-3) by the path recursion ---------------
   if (set == 0 && live) {
     const int d = ms.dep[n];
-    if (is_q) row_coefficients<true, kGdn>(sm, paths, ms, n, d, n);
-    else row_coefficients<false, kGdn>(sm, paths, ms, n, d, kTile + n);
+    if (fast) {
+      if (is_q) row_coefficients<true, kGdn>(sm, paths, ms, n, d, n);
+      else row_coefficients<false, kGdn>(sm, paths, ms, n, d, kTile + n);
+    } else {
+      if (is_q) row_coefficients_deep<true, kGdn>(sm, paths, ms, n, d, n);
+      else row_coefficients_deep<false, kGdn>(sm, paths, ms, n, d, kTile + n);
+    }
   }
   ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
@@ -466,6 +505,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
   release_tmem(warp, tmem);
+  // coalesced rows: a warp writes one 512-byte row of o or U per instruction
   Tout *out = static_cast<Tout *>(a.out);
   const int v4 = lane * 4;
   for (int r = warp; r < 2 * n_nodes; r += kThreads / 32) {
@@ -525,7 +565,11 @@ cudaError_t launch_tc_t(const VerifyArgs &a, cudaStream_t st) {
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<a.B * a.H, kThreads, kSmemBytes, st>>>(mq, mk, mv, a);
+  // the CTA one resident wave ahead (two per SM) gets its inputs prefetched into L2
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  kern<<<a.B * a.H, kThreads, kSmemBytes, st>>>(mq, mk, mv, a, 2 * sms);
   return cudaGetLastError();
 }
 
