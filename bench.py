@@ -335,7 +335,7 @@ def run_b200(args, workloads):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * max_s / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16xbf16->f32" if tc else "f32", "data": "synthetic",
+            "dtype": "bf16/tf32 tensor, f32 accumulate" if tc else "f32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "B": B, "H": H, "nodes_per_tree": 64,
                        "dk": w0.dk, "dv": w0.dv, "seeds": list(range(N_SETS)),
                        "l2": f"{N_SETS} rotating input sets, {N_SETS}x{vb / 1e6:.0f} MB > 126 MB L2",
@@ -358,10 +358,10 @@ def run_b200(args, workloads):
             "clocks": clk,
         }
         if world == 1 and not args.no_cpu_baseline:
-            n, dt = oracle_nodes(workloads[0], list(range(4 * 64)))
+            n, dt = oracle_nodes(workloads[0], list(range(10 * 64)))
             line["cpu_baseline"] = {
                 "value": n / dt, "unit": "nodes/s", "cores": 1, "kind": "oracle",
-                "sample": "sequences 0-3 (4 x 64 nodes x 32 heads) of the workload, verify + "
+                "sample": "sequences 0-9 (10 x 64 nodes x 32 heads) of the workload, verify + "
                           "commit, fp64 numpy, one BLAS thread", "seconds": dt}
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -374,7 +374,7 @@ def run_b200(args, workloads):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=10000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--kernel", choices=["auto", "tc", "simt"], default="auto")
