@@ -293,21 +293,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       ptx::mma_commit(bar_mma1);
     }
   }
-  if (tid == kThreads - 32) {
-    // L2 prefetch for the CTA one resident wave ahead: its S_root block and q / k / v tiles
-    const int nxt = blockIdx.x + prefetch_stride;
-    if (nxt < a.B * H) {
-      const int s2 = nxt / H, h2 = nxt % H;
-      ptx::prefetch_l2(a.S_root + (size_t)nxt * 128 * 128, 128 * 128 * 4);
-      const int lo2 = a.node_offsets[s2];
-      if (lo2 >= 0 && lo2 < a.T)
-        for (int half = 0; half < 2; ++half) {
-          ptx::prefetch_tile_l2(&tm_q, half * 64, h2, lo2);
-          ptx::prefetch_tile_l2(&tm_k, half * 64, h2, lo2);
-          ptx::prefetch_tile_l2(&tm_v, half * 64, h2, lo2);
-        }
-    }
-  }
   if (tid < kTile) {
     // ancestors in ascending index order are the root-first path; cl summed in that order
     unsigned long long bits = 0ull;
@@ -353,6 +338,23 @@ __global__ void __launch_bounds__(kThreads, 2)
   const bool fast = ms.maxdep <= kRegDepth;   // compact Gram entries, register recursion
 
   // ---- 3. accumulator 1 -> R (k lanes), gamma S_root q in place (q lanes), Gram ---------
+  if (tid == kThreads - 32) {
+    // L2 prefetch for the CTA one resident wave ahead: its S_root block and q / k / v
+    // tiles.  Issued once this CTA's own operands are consumed (MMA 1 done): earlier it
+    // competes with this CTA's loads, later it arrives too late for the next CTA.
+    const int nxt = blockIdx.x + prefetch_stride;
+    if (nxt < a.B * H) {
+      const int s2 = nxt / H, h2 = nxt % H;
+      ptx::prefetch_l2(a.S_root + (size_t)nxt * 128 * 128, 128 * 128 * 4);
+      const int lo2 = a.node_offsets[s2];
+      if (lo2 >= 0 && lo2 < a.T)
+        for (int half = 0; half < 2; ++half) {
+          ptx::prefetch_tile_l2(&tm_q, half * 64, h2, lo2);
+          ptx::prefetch_tile_l2(&tm_k, half * 64, h2, lo2);
+          ptx::prefetch_tile_l2(&tm_v, half * 64, h2, lo2);
+        }
+    }
+  }
   // warp w owns TMEM lanes 32*(w%4)..; warps 0-3 take value columns 0..63 and Gram
   // columns 0..31, warps 4-7 value columns 64..127 and Gram columns 32..63.
   const int quarter = warp & 3, set = warp >> 2;
