@@ -196,6 +196,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 }
 
 // Instruction descriptor: tf32 x tf32 -> fp32 (kind::tf32), both operands K-major.
+// D (+)= A . B^T, kind::tf32, A read from tensor memory (row m of A in lane m, K element k
+// in column a_tmem + k; 8 columns per instruction), B from a shared-memory descriptor.
+__device__ __forceinline__ void mma_tf32_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 __host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N) {
   return (1u << 4)                 // D format: fp32
          | (2u << 7)               // A format: tf32

@@ -5,13 +5,6 @@
 // strict ancestors anc(n) plus n (root first, indices increase along it), cl_n = fp32 sum
 // of log_a over path(n) (root first), gamma_n = exp(cl_n), D[n][i] = exp(cl_n - cl_i).
 //
-// MMA 1 (tcgen05 kind::f16, 128 x 192 x 128, bf16 in, fp32 accumulate in TMEM):
-//      [ Q ] . [ K ; S_root ]^T  ->  [ Q K^T | (S_root Q^T)^T ]   lanes 0..63
-//      [ K ]                         [ K K^T | (S_root K^T)^T ]   lanes 64..127
-// gives both path Gram blocks and both state products.  q, k, v arrive by TMA in the
-// 128-byte swizzled layout the MMA reads; S_root (fp32 in HBM) is converted to bf16 by all
-// threads straight into the same layout.
-//
 // The tree system (tree-structured WY form of the TreeWY abstract) is
 //      (I + L) U = R,  L[n][i] = b_n D[n][i] k_n.k_i (i in anc(n)),  R_n = b_n (v_n - gamma_n S_root k_n)
 // and the outputs (closed form of the Bole summary's worked example, "具体技术细节示例",
@@ -24,15 +17,28 @@
 //      omega_a = q_n.k_{p_a}                - sum_{c > a} omega_c b_{p_c} k_{p_c}.k_{p_a}
 // one thread per row, in registers.  Scalar decay: T = I (U = V), W = P.
 //
-// MMA 2 (kind::tf32, 128 x 128 x 64, operands rounded to nearest tf32) accumulates
-// [ W ; T ] . R onto accumulator columns 64..191, which by then hold gamma_n S_root q_n
-// (q lanes, rescaled in place) and zeros (k lanes): the accumulator ends as [ O ; U ].
-// It leaves through a swizzled shared tile as coalesced 512-byte rows.
+// The accumulator is kept transposed -- tensor-memory lane = value index, column = node --
+// so that R^T can be formed in place and fed back to the tensor core from tensor memory,
+// and so that every warp's output store is a contiguous 128-byte row segment.
+// Order of work in one CTA (one item; two CTAs per SM):
+//   1. the S_root loads (64 KiB) go out first, into registers; TMA brings q, k, v in the
+//      128-byte swizzled layout the MMA reads.
+//   2. Gram MMA (tcgen05 kind::f16, 128 x 64 x 128): [Q ; K] . K^T into columns 128..191,
+//      as soon as q and k have landed; meanwhile the tree is walked.
+//   3-4. Gram entries by path position, then the T and W row recursions -- none of which
+//      needs S_root, so they run while S_root is still arriving; then S_root -> bf16.
+//   5. state MMA (kind::f16, 128 x 128 x 128): S_root . [Q ; K]^T into columns 0..127.
+//   6. per value lane: columns 0..63 scaled by gamma_n; R^T[v][j] = b_j v_j[v] -
+//      b_j gamma_j (S_root k_j)[v] into columns 192..255 (tf32); [W ; T] written as the
+//      shared-memory operand.
+//   7. path-sum MMA (kind::tf32, A = R^T from tensor memory): columns 0..63 += R^T . W^T,
+//      columns 64..127 = R^T . T^T, i.e. o^T and U^T.
+//   8. tensor memory -> registers -> 128-byte row segments of o and U.
+// Trees deeper than kRegDepth take dense Gram matrices and an in-shared-memory recursion
+// in step 6 instead of steps 3-4.
 //
-// Two CTAs (about 104 KiB of shared memory each) share an SM so that one's loads overlap
-// the other's math.  Every wait on an mbarrier is bounded; a wait that runs out records
-// TV_ERR_TIMEOUT on the status word, the CTA drains what it issued, frees its tensor
-// memory and returns.
+// Every wait on an mbarrier is bounded; a wait that runs out records TV_ERR_TIMEOUT on
+// the status word, the CTA drains what it issued, frees its tensor memory and returns.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -45,57 +51,55 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kTile = 64;                  // nodes per tree handled by this kernel
-constexpr int kRegDepth = 8;               // deeper paths take the shared-memory recursion
-constexpr uint32_t kTmemCols = 256;        // accumulator columns 0..191; two CTAs per SM
+constexpr int kRegDepth = 8;               // deeper trees take the shared-memory recursion
+constexpr uint32_t kTmemCols = 256;        // two CTAs per SM
+constexpr uint32_t kColGram = 128;         // [Q ; K] . K^T  (lanes = q / k rows)
+constexpr uint32_t kColR = 192;            // R^T            (lanes = value index)
 constexpr uint32_t kSpinLimit = 1u << 22;  // polls before a wait is declared timed out
 
 // Dynamic shared memory, offsets from a 1024-byte aligned base.
-//   [0, 64K)    MMA 1 operands: two 64-wide K halves of [Q ; K ; S_root] (256 rows x 128 B)
-//               then  R^T (MMA 2 B operand, K-major, 128 x 64 fp32)       [0, 32K)
-//                     [W ; T] (MMA 2 A operand, K-major, 128 x 64 fp32)   [32K, 64K)
-//               then  O tile [0, 32K) and U tile [32K, 64K) (64 x 128 fp32 each)
-//   [64K, 80K)  v tile (bf16, TMA swizzled), then q_n.k_i on paths (64 x 64 fp32)
-//   [80K, 96K)  b_j k_j.k_i on paths (64 x 64 fp32)
-//   [96K, 100K) root-first paths, position-major bytes: node m's a-th entry at a*64 + m
-constexpr int kOpHalf = 256 * 128;
-constexpr int kOffOp = 0;
-constexpr int kOffB2 = 0;
-constexpr int kOffA2 = 32768;
-constexpr int kAtom2 = 16384;              // one 32-wide K atom of a 128-row MMA 2 operand
-constexpr int kOffOt = 0;
-constexpr int kOffUt = 32768;
+//   [0, 32K)    [Q ; K]: 128 rows x 128 bf16 as two 64-wide K halves of 16 KiB (TMA swizzled)
+//               then [W ; T]: path-sum B operand, 128 rows x 64 fp32, two 32-wide K atoms
+//   [32K, 64K)  S_root in bf16: 128 value rows x 128, two K halves
+//               then (deep trees) dense q_n.k_i [32K, 48K) and b_j k_j.k_i [48K, 64K)
+//   [64K, 80K)  v tile (bf16, TMA swizzled, two 64-wide value halves)
+//   [80K, 84K)  root-first paths, position-major bytes: node m's a-th entry at a*64 + m
+constexpr int kHalf = 128 * 128;           // one 64-wide K half of a 128-row bf16 operand
+constexpr int kOffQK = 0;
+constexpr int kOffA2 = 0;
+constexpr int kAtom2 = 16384;              // one 32-wide K atom of the 128-row fp32 operand
+constexpr int kOffS = 32768;
+constexpr int kOffGQ = 32768;
+constexpr int kOffLK = 49152;
 constexpr int kVHalf = kTile * 128;
 constexpr int kOffV = 65536;
-constexpr int kOffGQ = 65536;
-constexpr int kOffLK = 81920;
-constexpr int kOffPath = 98304;
+constexpr int kOffPath = 81920;
 constexpr int kOffMisc = kOffPath + kTile * kTile;
 
 struct Misc {
   unsigned long long bar_tma;
-  unsigned long long bar_mma1;
-  unsigned long long bar_mma2;
+  unsigned long long bar_gram;
+  unsigned long long bar_state;
+  unsigned long long bar_sum;
   unsigned long long anc[kTile];   // strict-ancestor bitmask
   uint32_t tmem_base;
-  int flag;                        // 0, or a tv_status to record for this item
+  int flag;                        // 0, or TV_ERR_TIMEOUT
   int maxdep;
-  // trees no deeper than kRegDepth keep the path Gram entries by path position:
+  // trees no deeper than kRegDepth, by path position:
   float lpos[kTile][kRegDepth];    // b_j k_j.k_{a-th ancestor of j}
-  float gpos[kTile][kRegDepth];    // q_n.k_{a-th node of path(n)}
+  float gpos[kTile][kRegDepth];    // q_n.k_{a-th node of path(n)}, then W[n][p_a]
+  float tpos[kTile][kRegDepth];    // T[n][p_a]
   int par[kTile];
   int dep[kTile];
   float la[kTile];
-  float bb[kTile];
+  float bb[kTile];                 // b_n
   float cl[kTile];
+  float gam[kTile];                // gamma_n
+  float bg[kTile];                 // b_n gamma_n
 };
 constexpr int kSmemBytes = kOffMisc + (int)sizeof(Misc) + 1024;
 
-// fp32 [64][128] tile in four 32-column slabs of 128-byte rows with 16-byte chunks
-// XOR-swizzled by row: row-per-thread writes and row-per-warp reads are conflict-free.
-__device__ __forceinline__ int tile_off(int n, int v) {
-  return ((v >> 5) << 13) + (n << 7) + ((((v >> 2) & 7) ^ (n & 7)) << 4) + ((v & 3) << 2);
-}
-// fp32 element (row, k) of a K-major MMA 2 operand (128 rows, K = 64, 128-byte swizzle).
+// fp32 element (row, k) of the K-major path-sum operand (128 rows, K = 64, 128-byte swizzle).
 __device__ __forceinline__ int op2_off(int row, int k) {
   return ((k >> 5) * kAtom2) + (row << 7) + ((((k >> 2) & 7) ^ (row & 7)) << 4) + ((k & 3) << 2);
 }
@@ -114,13 +118,58 @@ __device__ __forceinline__ float tf32_rn(float x) {
   asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
   return __uint_as_float(r);
 }
+// Streaming 16-byte load that stays where it is written: ahead of the tree-range check.
+__device__ __forceinline__ float4 ldg_first(const float4 *p) {
+  float4 r;
+  asm volatile("ld.global.cs.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+               : "l"(p));
+  return r;
+}
+__device__ __forceinline__ void st_out(float *p, float x) { __stcs(p, x); }
+__device__ __forceinline__ void st_out(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
 
-// Row m of [W ; T] (A2 row `r2`): x_a for path positions a < d,
-//   x_a = x0_a - sum_{c > a} x_c lk[p_c][p_a]   (x0 = e_{d-1}: T row; x0 = gq row: W row)
-// (no recursion for scalar decay, where L = 0), times D[m][p_a], rounded to tf32 and
-// stored at column p_a.  Trees deeper than kRegDepth run this in the A2 row itself on
-// dense Gram matrices, out of line so that the register version below (compact,
-// position-indexed Gram entries) stays small in the instruction cache.
+// One K = 128 chain of bf16 MMAs: D = A . B^T with A and B 128-row K-major operands.
+__device__ __forceinline__ void mma_chain_bf16(uint32_t a_base, uint32_t b_base, uint32_t d_tmem,
+                                               uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+    ptx::mma_bf16(d_tmem, ptx::smem_desc_sw128(a_base + off, 1024),
+                  ptx::smem_desc_sw128(b_base + off, 1024), idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// Row m, by path position a < d:  x_a = x0_a - sum_{c > a} x_c lpos[p_c][a]
+// (x0 = e_{d-1}: T row; x0 = gpos row: W row; no recursion for scalar decay), times
+// D[m][p_a], rounded to tf32, stored by position (tpos, or over gpos for W).
+template <bool kW, bool kGdn>
+__device__ __forceinline__ void row_coefficients(Misc &ms, const uint8_t *paths, int m, int d) {
+  const float clm = ms.cl[m];
+  int p[kRegDepth];
+  float x[kRegDepth];
+#pragma unroll
+  for (int a = 0; a < kRegDepth; ++a) {
+    p[a] = a < d ? paths[a * kTile + m] : m;
+    x[a] = kW ? (a < d ? ms.gpos[m][a] : 0.f) : (a == d - 1 ? 1.f : 0.f);
+  }
+#pragma unroll
+  for (int c = kRegDepth - 1; c >= 1; --c) {
+    if (kGdn && c < d) {
+      const float xc = x[c];
+#pragma unroll
+      for (int a = 0; a < c; ++a) x[a] = fmaf(-xc, ms.lpos[p[c]][a], x[a]);
+    }
+  }
+  float *dst = kW ? &ms.gpos[m][0] : &ms.tpos[m][0];
+#pragma unroll
+  for (int a = 0; a < kRegDepth; ++a)
+    if (a < d) dst[a] = tf32_rn(x[a] * __expf(clm - ms.cl[p[a]]));
+}
+
+// The same for trees deeper than kRegDepth, on dense Gram matrices, in the operand row
+// itself (node-indexed columns); out of line so that the register version stays small in
+// the instruction cache.
 template <bool kW, bool kGdn>
 __device__ __noinline__ void row_coefficients_deep(unsigned char *sm, const uint8_t *paths,
                                                    const Misc &ms, int m, int d, int r2) {
@@ -146,30 +195,6 @@ __device__ __noinline__ void row_coefficients_deep(unsigned char *sm, const uint
   }
 }
 
-template <bool kW, bool kGdn>
-__device__ __forceinline__ void row_coefficients(unsigned char *sm, const uint8_t *paths,
-                                                 const Misc &ms, int m, int d, int r2) {
-  const float clm = ms.cl[m];
-  int p[kRegDepth];
-  float x[kRegDepth];
-#pragma unroll
-  for (int a = 0; a < kRegDepth; ++a) {
-    p[a] = a < d ? paths[a * kTile + m] : m;
-    x[a] = kW ? (a < d ? ms.gpos[m][a] : 0.f) : (a == d - 1 ? 1.f : 0.f);
-  }
-#pragma unroll
-  for (int c = kRegDepth - 1; c >= 1; --c) {
-    if (kGdn && c < d) {
-      const float xc = x[c];
-#pragma unroll
-      for (int a = 0; a < c; ++a) x[a] = fmaf(-xc, ms.lpos[p[c]][a], x[a]);
-    }
-  }
-#pragma unroll
-  for (int a = 0; a < kRegDepth; ++a)
-    if (a < d) sts(sm, kOffA2 + op2_off(r2, p[a]), tf32_rn(x[a] * __expf(clm - ms.cl[p[a]])));
-}
-
 __device__ __forceinline__ void release_tmem(int warp, uint32_t tmem) {
   ptx::tc_fence_before();
   __syncthreads();
@@ -177,6 +202,18 @@ __device__ __forceinline__ void release_tmem(int warp, uint32_t tmem) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+// One thread waits on `bar`; every thread learns whether it completed.  On a time-out the
+// status is recorded, the wait is retried once (bounded) and the CTA must leave.
+__device__ __forceinline__ bool wait_all(Misc &ms, uint32_t bar, int tid, int *ws, int s) {
+  if (tid == 0 && !ptx::mbar_wait_bounded(bar, 0, kSpinLimit)) {
+    ms.flag = TV_ERR_TIMEOUT;
+    set_status(ws, TV_ERR_TIMEOUT, s);
+    ptx::mbar_wait_bounded(bar, 0, kSpinLimit);
+  }
+  __syncthreads();
+  return ms.flag == 0;
 }
 
 template <bool kGdn, typename Tout>
@@ -194,6 +231,20 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int H = a.H;
   const int s = blockIdx.x / H, h = blockIdx.x % H;
 
+  // ---- 1. S_root loads, the tree's node range, q / k / v by TMA, tree inputs ----------
+  // S_root as 16 float4 per thread: thread t owns 8-element k chunk (t & 15) of value rows
+  // t/16 + 16 j.  Issued before anything else; consumed in step 4.
+  const int kc = tid & 15;
+  float4 sr[16];
+  {
+    const float4 *Sg = reinterpret_cast<const float4 *>(a.S_root + ((size_t)s * H + h) * 128 * 128);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int v = (tid >> 4) + 16 * j;
+      sr[2 * j] = ldg_first(Sg + v * 32 + kc * 2);
+      sr[2 * j + 1] = ldg_first(Sg + v * 32 + kc * 2 + 1);
+    }
+  }
   const int lo = a.node_offsets[s], hi = a.node_offsets[s + 1];
   if (lo < 0 || hi < lo || hi > a.T || hi - lo > a.max_nodes || hi - lo > kTile ||
       (s == 0 && lo != 0) || (s == a.B - 1 && hi != a.T)) {
@@ -205,14 +256,14 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   const uint32_t sbase = ptx::smem_addr(sm);
   const uint32_t bar_tma = ptx::smem_addr(&ms.bar_tma);
-  const uint32_t bar_mma1 = ptx::smem_addr(&ms.bar_mma1);
-  const uint32_t bar_mma2 = ptx::smem_addr(&ms.bar_mma2);
-
-  // ---- 1. TMA of q / k / v, tensor memory, S_root -> bf16 operand rows 128..255 --------
+  const uint32_t bar_gram = ptx::smem_addr(&ms.bar_gram);
+  const uint32_t bar_state = ptx::smem_addr(&ms.bar_state);
+  const uint32_t bar_sum = ptx::smem_addr(&ms.bar_sum);
   if (tid == 0) {
     ptx::mbar_init(bar_tma, 1);
-    ptx::mbar_init(bar_mma1, 1);
-    ptx::mbar_init(bar_mma2, 1);
+    ptx::mbar_init(bar_gram, 1);
+    ptx::mbar_init(bar_state, 1);
+    ptx::mbar_init(bar_sum, 1);
     ptx::fence_mbar_init();
     ms.flag = 0;
     ms.maxdep = 0;
@@ -221,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     ptx::prefetch_tmap(&tm_v);
     ptx::mbar_arrive_expect_tx(bar_tma, 6 * kTile * 128);
     for (int half = 0; half < 2; ++half) {
-      const uint32_t hb = sbase + kOffOp + half * kOpHalf;
+      const uint32_t hb = sbase + kOffQK + half * kHalf;
       ptx::tma_load_3d(hb, &tm_q, bar_tma, half * 64, h, lo);
       ptx::tma_load_3d(hb + kTile * 128, &tm_k, bar_tma, half * 64, h, lo);
       ptx::tma_load_3d(sbase + kOffV + half * kVHalf, &tm_v, bar_tma, half * 64, h, lo);
@@ -232,65 +283,33 @@ __global__ void __launch_bounds__(kThreads, 2)
     ptx::tmem_relinquish();
   }
   bool bad = false;
-  {
-    const float4 *Sg = reinterpret_cast<const float4 *>(a.S_root + ((size_t)s * H + h) * 128 * 128);
-    const int kc = tid & 15;                 // 8-element chunk of k owned by this thread
-    float4 r[16];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int v = (tid >> 4) + 16 * j;
-      r[2 * j] = __ldcs(Sg + v * 32 + kc * 2);
-      r[2 * j + 1] = __ldcs(Sg + v * 32 + kc * 2 + 1);
+  if (tid < kTile) {
+    int p = -1;
+    float la = 0.f, bb = 0.f;
+    if (tid < n_nodes) {
+      p = a.parent[lo + tid];
+      bad = p < -1 || p >= tid;
+      la = a.log_a[(size_t)(lo + tid) * H + h];
+      bb = kGdn ? a.b[(size_t)(lo + tid) * H + h] : 0.f;
     }
-    if (tid < kTile) {
-      int p = -1;
-      float la = 0.f, bb = 0.f;
-      if (tid < n_nodes) {
-        p = a.parent[lo + tid];
-        bad = p < -1 || p >= tid;
-        la = a.log_a[(size_t)(lo + tid) * H + h];
-        bb = kGdn ? a.b[(size_t)(lo + tid) * H + h] : 0.f;
-      }
-      ms.par[tid] = p;
-      ms.la[tid] = la;
-      ms.bb[tid] = bb;
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int v = (tid >> 4) + 16 * j, row = 128 + v;
-      __nv_bfloat162 b0 = __floats2bfloat162_rn(r[2 * j].x, r[2 * j].y);
-      __nv_bfloat162 b1 = __floats2bfloat162_rn(r[2 * j].z, r[2 * j].w);
-      __nv_bfloat162 b2 = __floats2bfloat162_rn(r[2 * j + 1].x, r[2 * j + 1].y);
-      __nv_bfloat162 b3 = __floats2bfloat162_rn(r[2 * j + 1].z, r[2 * j + 1].w);
-      uint4 pk;
-      pk.x = *reinterpret_cast<uint32_t *>(&b0);
-      pk.y = *reinterpret_cast<uint32_t *>(&b1);
-      pk.z = *reinterpret_cast<uint32_t *>(&b2);
-      pk.w = *reinterpret_cast<uint32_t *>(&b3);
-      const int off = (kc >> 3) * kOpHalf + row * 128 + (((kc & 7) ^ (row & 7)) << 4);
-      *reinterpret_cast<uint4 *>(sm + kOffOp + off) = pk;
-    }
-    ptx::fence_proxy_async_smem();
+    ms.par[tid] = p;
+    ms.la[tid] = la;
+    ms.bb[tid] = bb;
   }
   ptx::tc_fence_before();
   const bool bad_tree = __syncthreads_or(bad) != 0;
   ptx::tc_fence_after();
   const uint32_t tmem = ms.tmem_base;
 
-  // ---- 2. MMA 1 (one thread) while the tree metadata is formed -------------------------
+  // ---- 2. Gram MMA once q / k have landed; tree walk ------------------------------------
   if (tid == kThreads - 1) {
     if (!ptx::mbar_wait_bounded(bar_tma, 0, kSpinLimit)) {
       ms.flag = TV_ERR_TIMEOUT;
     } else if (!bad_tree) {
       ptx::tc_fence_after();
-      constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, 192);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t base = sbase + kOffOp + (kk >> 2) * kOpHalf + (kk & 3) * 32;
-        ptx::mma_bf16(tmem, ptx::smem_desc_sw128(base, 1024),
-                      ptx::smem_desc_sw128(base + kTile * 128, 1024), idesc, kk > 0 ? 1u : 0u);
-      }
-      ptx::mma_commit(bar_mma1);
+      mma_chain_bf16(sbase + kOffQK, sbase + kOffQK + kTile * 128, tmem + kColGram,
+                     ptx::idesc_bf16_f32(128, 64));
+      ptx::mma_commit(bar_gram);
     }
   }
   if (tid < kTile) {
@@ -310,9 +329,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       cl += ms.la[tid];
       ++d;
     }
+    const float gam = __expf(cl);
     ms.anc[tid] = bits;
     ms.dep[tid] = d;
     ms.cl[tid] = cl;
+    ms.gam[tid] = gam;
+    ms.bg[tid] = ms.bb[tid] * gam;
     atomicMax(&ms.maxdep, d);
   }
   __syncthreads();
@@ -324,24 +346,87 @@ __global__ void __launch_bounds__(kThreads, 2)
     release_tmem(warp, tmem);
     return;
   }
-  if (tid == 0 && !ptx::mbar_wait_bounded(bar_mma1, 0, kSpinLimit)) ms.flag = TV_ERR_TIMEOUT;
-  __syncthreads();
-  if (ms.flag != 0) {
-    if (tid == 0) {
-      set_status(a.ws, ms.flag, s);
-      ptx::mbar_wait_bounded(bar_mma1, 0, kSpinLimit);
-    }
+  if (!wait_all(ms, bar_gram, tid, a.ws, s)) {
     release_tmem(warp, tmem);
     return;
   }
   ptx::tc_fence_after();
-  const bool fast = ms.maxdep <= kRegDepth;   // compact Gram entries, register recursion
+  const bool fast = ms.maxdep <= kRegDepth;
 
-  // ---- 3. accumulator 1 -> R (k lanes), gamma S_root q in place (q lanes), Gram ---------
+  // warp w reads tensor-memory lanes 32*(w%4)..; `set` = w/4 splits the columns in two.
+  const int quarter = warp & 3, set = warp >> 2;
+  const uint32_t tlane = tmem + ((uint32_t)(quarter * 32) << 16);
+  // in the Gram columns, lane r is row r of [Q ; K]
+  const int grow = quarter * 32 + lane;
+  const bool g_is_q = grow < kTile;
+  const int gn = grow & (kTile - 1);
+  const bool g_live = gn < n_nodes;
+
+  // ---- 3. Gram entries by path position: k rows b_n k_n.k_i on anc(n), q rows q_n.k_i on
+  // path(n) (a node's position on a path = the number of path nodes with a smaller index)
+  if (fast && (g_is_q || kGdn)) {
+    const unsigned long long ancn = ms.anc[gn];
+    const unsigned long long sel = !g_live ? 0ull : (g_is_q ? (ancn | (1ull << gn)) : ancn);
+    const float scale = g_is_q ? 1.f : ms.bb[gn];
+    float *posrow = g_is_q ? &ms.gpos[gn][0] : &ms.lpos[gn][0];
+#pragma unroll 1
+    for (int c = 0; c < 2; ++c) {
+      float g[16];
+      const int i0 = set * 32 + c * 16;
+      ptx::tmem_ld16(tlane + kColGram + i0, g);
+      const unsigned bits = (unsigned)(sel >> i0) & 0xFFFFu;
+      int pos = __popcll(sel & ((1ull << i0) - 1ull));
+      ptx::tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if ((bits >> j) & 1u) posrow[pos++] = scale * g[j];
+    }
+  }
+  __syncthreads();
+
+  // ---- 4. T and W rows (shallow trees, warps 0-3) while S_root arrives; S_root -> bf16 --
+  if (fast && tid < 2 * kTile) {
+    const int m = tid & (kTile - 1);
+    if (m < n_nodes) {
+      const int d = ms.dep[m];
+      if (tid < kTile) row_coefficients<true, kGdn>(ms, paths, m, d);
+      else row_coefficients<false, kGdn>(ms, paths, m, d);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int v = (tid >> 4) + 16 * j;
+    __nv_bfloat162 b0 = __floats2bfloat162_rn(sr[2 * j].x, sr[2 * j].y);
+    __nv_bfloat162 b1 = __floats2bfloat162_rn(sr[2 * j].z, sr[2 * j].w);
+    __nv_bfloat162 b2 = __floats2bfloat162_rn(sr[2 * j + 1].x, sr[2 * j + 1].y);
+    __nv_bfloat162 b3 = __floats2bfloat162_rn(sr[2 * j + 1].z, sr[2 * j + 1].w);
+    uint4 pk;
+    pk.x = *reinterpret_cast<uint32_t *>(&b0);
+    pk.y = *reinterpret_cast<uint32_t *>(&b1);
+    pk.z = *reinterpret_cast<uint32_t *>(&b2);
+    pk.w = *reinterpret_cast<uint32_t *>(&b3);
+    const int off = (kc >> 3) * kHalf + v * 128 + (((kc & 7) ^ (v & 7)) << 4);
+    *reinterpret_cast<uint4 *>(sm + kOffS + off) = pk;
+  }
+  ptx::fence_proxy_async_smem();
+  ptx::tc_fence_before();
+  __syncthreads();
+
+  // ---- 5. state MMA: columns 0..127 = S_root . [Q ; K]^T ------------------------------------
+  if (tid == kThreads - 1) {
+    ptx::tc_fence_after();
+    mma_chain_bf16(sbase + kOffS, sbase + kOffQK, tmem, ptx::idesc_bf16_f32(128, 128));
+    ptx::mma_commit(bar_state);
+  }
+  if (!wait_all(ms, bar_state, tid, a.ws, s)) {
+    release_tmem(warp, tmem);
+    return;
+  }
+  ptx::tc_fence_after();
   if (tid == kThreads - 32) {
     // L2 prefetch for the CTA one resident wave ahead: its S_root block and q / k / v
-    // tiles.  Issued once this CTA's own operands are consumed (MMA 1 done): earlier it
-    // competes with this CTA's loads, later it arrives too late for the next CTA.
+    // tiles.  Issued once this CTA's own operands are consumed: earlier it competes with
+    // this CTA's loads, later it arrives too late for the next CTA.
     const int nxt = blockIdx.x + prefetch_stride;
     if (nxt < a.B * H) {
       const int s2 = nxt / H, h2 = nxt % H;
@@ -355,176 +440,132 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
     }
   }
-  // warp w owns TMEM lanes 32*(w%4)..; warps 0-3 take value columns 0..63 and Gram
-  // columns 0..31, warps 4-7 value columns 64..127 and Gram columns 32..63.
-  const int quarter = warp & 3, set = warp >> 2;
-  const int row = quarter * 32 + lane;
-  const bool is_q = row < kTile;
-  const int n = is_q ? row : row - kTile;
-  const bool live = n < n_nodes;
-  const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
-  const unsigned long long ancn = ms.anc[n];
+
+  // ---- 6. [W ; T] operand over the dead [Q ; K] tile; gamma o^T and R^T in tensor memory --
   {
-    const float gam = __expf(ms.cl[n]);
-    const float bn = ms.bb[n];
-    const unsigned char *vt = sm + kOffV;
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      float x[16];
-      const int v0 = set * 64 + c * 16;
-      ptx::tmem_ld16(trow + 64 + v0, x);
-      if (is_q) {
-        ptx::tmem_wait_ld();
+    // thread t writes K atom t/128 of operand row t%128: zeros, then its path coefficients
+    const int r2 = tid & 127, atom = tid >> 7;
+    const float4 zf = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) x[j] *= gam;
-        ptx::tmem_st16(trow + 64 + v0, x);
-      } else {
-        const int half = v0 >> 6, ch = (v0 & 63) >> 3;
-        const uint4 w0 = *reinterpret_cast<const uint4 *>(
-            vt + half * kVHalf + (n << 7) + ((ch ^ (n & 7)) << 4));
-        const uint4 w1 = *reinterpret_cast<const uint4 *>(
-            vt + half * kVHalf + (n << 7) + (((ch + 1) ^ (n & 7)) << 4));
-        const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        ptx::tmem_wait_ld();
-        const float bg = bn * gam;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float vn = __uint_as_float(((wv[j >> 1] >> ((j & 1) * 16)) & 0xFFFFu) << 16);
-          x[j] = live ? tf32_rn(kGdn ? fmaf(-bg, x[j], bn * vn) : vn) : 0.f;
-        }
-        // column n of R^T: a warp's 32 nodes fill one 128-byte swizzle row per value v
-#pragma unroll
-        for (int j = 0; j < 16; ++j) sts(sm, kOffB2 + op2_off(v0 + j, n), x[j]);
-        float z[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) z[j] = 0.f;
-        ptx::tmem_st16(trow + 64 + v0, z);
+    for (int c = 0; c < 8; ++c)
+      *reinterpret_cast<float4 *>(sm + kOffA2 + op2_off(r2, atom * 32 + c * 4)) = zf;
+    const int n2 = r2 & (kTile - 1);
+    if (fast && n2 < n_nodes) {
+      const int d = ms.dep[n2];
+      const float *cf = r2 < kTile ? &ms.gpos[n2][0] : &ms.tpos[n2][0];
+      for (int a2 = 0; a2 < d; ++a2) {
+        const int i = paths[a2 * kTile + n2];
+        if ((i >> 5) == atom) sts(sm, kOffA2 + op2_off(r2, i), cf[a2]);
       }
     }
-    // Gram entries: k lanes b_n k_n.k_i on anc(n) (gated delta only); q lanes (compact
-    // form only) q_n.k_i on path(n).  Position of node i on a path = ancestors below i.
-    if (is_q ? fast : kGdn) {
-      const unsigned long long sel = !live ? 0ull : (is_q ? (ancn | (1ull << n)) : ancn);
-      const float scale = is_q ? 1.f : bn;
-      float *posrow = is_q ? &ms.gpos[n][0] : &ms.lpos[n][0];
+  }
+  if (!fast) {
+    // deep trees: dense q_n.k_i and b_n k_n.k_i over the dead S_root tile, then the row
+    // recursion in the operand rows (zero-filled above)
+    if (g_is_q || kGdn) {
+      const unsigned long long ancn = ms.anc[gn];
+      const unsigned long long sel = !g_live ? 0ull : (g_is_q ? (ancn | (1ull << gn)) : ancn);
+      const float scale = g_is_q ? 1.f : ms.bb[gn];
+      const int base = g_is_q ? kOffGQ : kOffLK;
 #pragma unroll 1
       for (int c = 0; c < 2; ++c) {
         float g[16];
         const int i0 = set * 32 + c * 16;
-        ptx::tmem_ld16(trow + i0, g);
-        const unsigned bits = (unsigned)(sel >> i0) & 0xFFFFu;
-        int pos = __popcll(sel & ((1ull << i0) - 1ull));   // path position of column i0
+        ptx::tmem_ld16(tlane + kColGram + i0, g);
         ptx::tmem_wait_ld();
-        if (!fast) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if ((bits >> j) & 1u) sts(sm, kOffLK + coef_off(n, i0 + j), scale * g[j]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if ((bits >> j) & 1u) posrow[pos++] = scale * g[j];
-        }
+        for (int j = 0; j < 16; ++j)
+          if ((sel >> (i0 + j)) & 1ull) sts(sm, base + coef_off(gn, i0 + j), scale * g[j]);
       }
     }
-    // [W ; T] starts as zeros
-    const float4 zf = make_float4(0.f, 0.f, 0.f, 0.f);
+    __syncthreads();
+    if (set == 0 && g_live) {
+      const int d = ms.dep[gn];
+      if (g_is_q) row_coefficients_deep<true, kGdn>(sm, paths, ms, gn, d, gn);
+      else row_coefficients_deep<false, kGdn>(sm, paths, ms, gn, d, kTile + gn);
+    }
+  }
+  {
+    // lane v of columns [32 set, 32 set + 32) (o) and [64 + 32 set, ...) (S_root k_j)
+    const int v = quarter * 32 + lane, j0 = set * 32;
+    float o0[16], o1[16], k0[16], k1[16];
+    ptx::tmem_ld16(tlane + j0, o0);
+    ptx::tmem_ld16(tlane + j0 + 16, o1);
+    ptx::tmem_ld16(tlane + kTile + j0, k0);
+    ptx::tmem_ld16(tlane + kTile + j0 + 16, k1);
+    ptx::tmem_wait_ld();
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      *reinterpret_cast<float4 *>(sm + kOffA2 + (tid + j * kThreads) * 16) = zf;
+    for (int j = 0; j < 16; ++j) {
+      o0[j] *= ms.gam[j0 + j];
+      o1[j] *= ms.gam[j0 + 16 + j];
+    }
+    ptx::tmem_st16(tlane + j0, o0);
+    ptx::tmem_st16(tlane + j0 + 16, o1);
+    // v_j[v]: value half v/64 of node j's row in the v tile
+    const unsigned char *vt = sm + kOffV + (v >> 6) * kVHalf + (v & 7) * 2;
+    const int vc = (v & 63) >> 3;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int ja = j0 + j, jb = j0 + 16 + j;
+      const float va = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(vt + ja * 128 + ((vc ^ (ja & 7)) << 4)));
+      const float vb = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(vt + jb * 128 + ((vc ^ (jb & 7)) << 4)));
+      k0[j] = ja < n_nodes ? tf32_rn(kGdn ? fmaf(-ms.bg[ja], k0[j], ms.bb[ja] * va) : va) : 0.f;
+      k1[j] = jb < n_nodes ? tf32_rn(kGdn ? fmaf(-ms.bg[jb], k1[j], ms.bb[jb] * vb) : vb) : 0.f;
+    }
+    ptx::tmem_st16(tlane + kColR + j0, k0);
+    ptx::tmem_st16(tlane + kColR + j0 + 16, k1);
   }
   ptx::tmem_wait_st();
-  ptx::tc_fence_before();
-  __syncthreads();
-  if (!fast) {
-  if (is_q) {   // dense q_n.k_i on path(n), into the now free v tile
-    ptx::tc_fence_after();
-    const unsigned long long sel = live ? (ancn | (1ull << n)) : 0ull;
-#pragma unroll 1
-    for (int c = 0; c < 2; ++c) {
-      float g[16];
-      const int i0 = set * 32 + c * 16;
-      ptx::tmem_ld16(trow + i0, g);
-      ptx::tmem_wait_ld();
-#pragma unroll
-      for (int j = 0; j < 16; ++j)
-        if ((sel >> (i0 + j)) & 1ull) sts(sm, kOffGQ + coef_off(n, i0 + j), g[j]);
-    }
-  }
-  __syncthreads();
-  }
-
-  // ---- 4. rows of W (warps 0-1) and T (warps 2-3) by the path recursion ---------------
-  if (set == 0 && live) {
-    const int d = ms.dep[n];
-    if (fast) {
-      if (is_q) row_coefficients<true, kGdn>(sm, paths, ms, n, d, n);
-      else row_coefficients<false, kGdn>(sm, paths, ms, n, d, kTile + n);
-    } else {
-      if (is_q) row_coefficients_deep<true, kGdn>(sm, paths, ms, n, d, n);
-      else row_coefficients_deep<false, kGdn>(sm, paths, ms, n, d, kTile + n);
-    }
-  }
   ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
   __syncthreads();
 
-  // ---- 5. MMA 2: accumulator columns 64..191 += [W ; T] . R  (tf32) --------------------
+  // ---- 7. path-sum MMA: columns 0..63 += R^T . W^T, columns 64..127 = R^T . T^T (tf32) ---
   if (tid == kThreads - 1) {
     ptx::tc_fence_after();
-    constexpr uint32_t idesc = ptx::idesc_tf32_f32(128, 128);
+    constexpr uint32_t idesc = ptx::idesc_tf32_f32(128, 64);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
-      const uint32_t koff = (kk >> 2) * kAtom2 + (kk & 3) * 32;
-      ptx::mma_tf32(tmem + 64, ptx::smem_desc_sw128(sbase + kOffA2 + koff, 1024),
-                    ptx::smem_desc_sw128(sbase + kOffB2 + koff, 1024), idesc, 1u);
+      const uint32_t kb = sbase + kOffA2 + (kk >> 2) * kAtom2 + (kk & 3) * 32;
+      const uint32_t ra = tmem + kColR + kk * 8;
+      ptx::mma_tf32_tmem_a(tmem, ra, ptx::smem_desc_sw128(kb, 1024), idesc, 1u);
+      ptx::mma_tf32_tmem_a(tmem + kTile, ra, ptx::smem_desc_sw128(kb + kTile * 128, 1024), idesc,
+                           kk > 0 ? 1u : 0u);
     }
-    ptx::mma_commit(bar_mma2);
+    ptx::mma_commit(bar_sum);
   }
-  if (tid == 0 && !ptx::mbar_wait_bounded(bar_mma2, 0, kSpinLimit)) ms.flag = TV_ERR_TIMEOUT;
-  __syncthreads();
-  if (ms.flag != 0) {
-    if (tid == 0) {
-      set_status(a.ws, ms.flag, s);
-      ptx::mbar_wait_bounded(bar_mma2, 0, kSpinLimit);
-    }
+  if (!wait_all(ms, bar_sum, tid, a.ws, s)) {
     release_tmem(warp, tmem);
     return;
   }
   ptx::tc_fence_after();
 
-  // ---- 6. accumulator -> O / U tiles -> coalesced rows ---------------------------------
+  // ---- 8. o^T and U^T -> 128-byte row segments (a warp's 32 lanes are 32 adjacent v) -----
   {
-    unsigned char *tile = sm + (is_q ? kOffOt : kOffUt);
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      float y[16];
-      const int v0 = set * 64 + c * 16;
-      ptx::tmem_ld16(trow + 64 + v0, y);
-      ptx::tmem_wait_ld();
+    const int v = quarter * 32 + lane, j0 = set * 32;
+    float o0[16], o1[16], u0[16], u1[16];
+    ptx::tmem_ld16(tlane + j0, o0);
+    ptx::tmem_ld16(tlane + j0 + 16, o1);
+    ptx::tmem_ld16(tlane + kTile + j0, u0);
+    ptx::tmem_ld16(tlane + kTile + j0 + 16, u1);
+    ptx::tmem_wait_ld();
+    release_tmem(warp, tmem);
+    Tout *out = static_cast<Tout *>(a.out) + ((size_t)lo * H + h) * 128 + v;
+    float *U = a.U + ((size_t)lo * H + h) * 128 + v;
+    const size_t rs = (size_t)H * 128;
 #pragma unroll
-      for (int j = 0; j < 16; j += 4)
-        *reinterpret_cast<float4 *>(tile + tile_off(n, v0 + j)) = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
+    for (int j = 0; j < 16; ++j) {
+      if (j0 + j < n_nodes) {
+        st_out(out + (j0 + j) * rs, o0[j]);
+        __stcs(U + (j0 + j) * rs, u0[j]);
+      }
     }
-  }
-  release_tmem(warp, tmem);
-  // coalesced rows: a warp writes one 512-byte row of o or U per instruction
-  Tout *out = static_cast<Tout *>(a.out);
-  const int v4 = lane * 4;
-  for (int r = warp; r < 2 * n_nodes; r += kThreads / 32) {
-    const bool is_u = r >= n_nodes;
-    const int m = is_u ? r - n_nodes : r;
-    const float4 x = *reinterpret_cast<const float4 *>(sm + (is_u ? kOffUt : kOffOt) + tile_off(m, v4));
-    const size_t g = ((size_t)(lo + m) * H + h) * 128 + v4;
-    if (is_u) {
-      __stcs(reinterpret_cast<float4 *>(a.U + g), x);
-    } else if (sizeof(Tout) == 4) {
-      __stcs(reinterpret_cast<float4 *>(reinterpret_cast<float *>(out) + g), x);
-    } else {
-      __nv_bfloat162 l2 = __floats2bfloat162_rn(x.x, x.y), h2 = __floats2bfloat162_rn(x.z, x.w);
-      uint2 pk;
-      pk.x = *reinterpret_cast<uint32_t *>(&l2);
-      pk.y = *reinterpret_cast<uint32_t *>(&h2);
-      *reinterpret_cast<uint2 *>(reinterpret_cast<__nv_bfloat16 *>(out) + g) = pk;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (j0 + 16 + j < n_nodes) {
+        st_out(out + (j0 + 16 + j) * rs, o1[j]);
+        __stcs(U + (j0 + 16 + j) * rs, u1[j]);
+      }
     }
   }
 }
