@@ -31,8 +31,8 @@
 //   6. per value lane: columns 0..63 scaled by gamma_n; R^T[v][j] = b_j v_j[v] -
 //      b_j gamma_j (S_root k_j)[v] into columns 192..255 (tf32); [W ; T] written as the
 //      shared-memory operand.
-//   7. path-sum MMA (kind::tf32, A = R^T from tensor memory): columns 0..63 += R^T . W^T,
-//      columns 64..127 = R^T . T^T, i.e. o^T and U^T.
+//   7. path-sum MMA (kind::tf32, A = R^T from tensor memory): columns 0..127 (o part
+//      rescaled, U part zeroed in step 6) += R^T . [W ; T]^T, i.e. o^T and U^T.
 //   8. tensor memory -> registers -> 128-byte row segments of o and U.
 // Trees deeper than kRegDepth take dense Gram matrices and an in-shared-memory recursion
 // in step 6 instead of steps 3-4.
@@ -85,17 +85,19 @@ struct Misc {
   uint32_t tmem_base;
   int flag;                        // 0, or TV_ERR_TIMEOUT
   int maxdep;
-  // trees no deeper than kRegDepth, by path position:
-  float lpos[kTile][kRegDepth];    // b_j k_j.k_{a-th ancestor of j}
-  float gpos[kTile][kRegDepth];    // q_n.k_{a-th node of path(n)}, then W[n][p_a]
-  float tpos[kTile][kRegDepth];    // T[n][p_a]
+  // trees no deeper than kRegDepth, position-major ([a][node]: a row-per-thread access
+  // touches 32 consecutive words):
+  float lpos[kRegDepth][kTile];    // b_j k_j.k_{a-th ancestor of j}
+  float gpos[kRegDepth][kTile];    // q_n.k_{a-th node of path(n)}, then W[n][p_a]
+  float tpos[kRegDepth][kTile];    // T[n][p_a]
   int par[kTile];
   int dep[kTile];
   float la[kTile];
   float bb[kTile];                 // b_n
   float cl[kTile];
-  float gam[kTile];                // gamma_n
-  float bg[kTile];                 // b_n gamma_n
+  __align__(16) float gam[kTile];  // gamma_n
+  __align__(16) float bg[kTile];   // b_n gamma_n
+  __align__(16) float bq[kTile];   // b_n (copy read as float4)
 };
 constexpr int kSmemBytes = kOffMisc + (int)sizeof(Misc) + 1024;
 
@@ -151,20 +153,20 @@ __device__ __forceinline__ void row_coefficients(Misc &ms, const uint8_t *paths,
 #pragma unroll
   for (int a = 0; a < kRegDepth; ++a) {
     p[a] = a < d ? paths[a * kTile + m] : m;
-    x[a] = kW ? (a < d ? ms.gpos[m][a] : 0.f) : (a == d - 1 ? 1.f : 0.f);
+    x[a] = kW ? (a < d ? ms.gpos[a][m] : 0.f) : (a == d - 1 ? 1.f : 0.f);
   }
 #pragma unroll
   for (int c = kRegDepth - 1; c >= 1; --c) {
     if (kGdn && c < d) {
       const float xc = x[c];
 #pragma unroll
-      for (int a = 0; a < c; ++a) x[a] = fmaf(-xc, ms.lpos[p[c]][a], x[a]);
+      for (int a = 0; a < c; ++a) x[a] = fmaf(-xc, ms.lpos[a][p[c]], x[a]);
     }
   }
-  float *dst = kW ? &ms.gpos[m][0] : &ms.tpos[m][0];
+  float(*dst)[kTile] = kW ? ms.gpos : ms.tpos;
 #pragma unroll
   for (int a = 0; a < kRegDepth; ++a)
-    if (a < d) dst[a] = tf32_rn(x[a] * __expf(clm - ms.cl[p[a]]));
+    if (a < d) dst[a][m] = tf32_rn(x[a] * __expf(clm - ms.cl[p[a]]));
 }
 
 // The same for trees deeper than kRegDepth, on dense Gram matrices, in the operand row
@@ -335,6 +337,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     ms.cl[tid] = cl;
     ms.gam[tid] = gam;
     ms.bg[tid] = ms.bb[tid] * gam;
+    ms.bq[tid] = ms.bb[tid];
     atomicMax(&ms.maxdep, d);
   }
   __syncthreads();
@@ -368,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const unsigned long long ancn = ms.anc[gn];
     const unsigned long long sel = !g_live ? 0ull : (g_is_q ? (ancn | (1ull << gn)) : ancn);
     const float scale = g_is_q ? 1.f : ms.bb[gn];
-    float *posrow = g_is_q ? &ms.gpos[gn][0] : &ms.lpos[gn][0];
+    float(*pos_major)[kTile] = g_is_q ? ms.gpos : ms.lpos;
 #pragma unroll 1
     for (int c = 0; c < 2; ++c) {
       float g[16];
@@ -379,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       ptx::tmem_wait_ld();
 #pragma unroll
       for (int j = 0; j < 16; ++j)
-        if ((bits >> j) & 1u) posrow[pos++] = scale * g[j];
+        if ((bits >> j) & 1u) pos_major[pos++][gn] = scale * g[j];
     }
   }
   __syncthreads();
@@ -452,10 +455,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int n2 = r2 & (kTile - 1);
     if (fast && n2 < n_nodes) {
       const int d = ms.dep[n2];
-      const float *cf = r2 < kTile ? &ms.gpos[n2][0] : &ms.tpos[n2][0];
-      for (int a2 = 0; a2 < d; ++a2) {
+      const float(*cf)[kTile] = r2 < kTile ? ms.gpos : ms.tpos;
+#pragma unroll
+      for (int a2 = 0; a2 < kRegDepth; ++a2) {
         const int i = paths[a2 * kTile + n2];
-        if ((i >> 5) == atom) sts(sm, kOffA2 + op2_off(r2, i), cf[a2]);
+        if (a2 < d && (i >> 5) == atom) sts(sm, kOffA2 + op2_off(r2, i), cf[a2][n2]);
       }
     }
   }
@@ -493,11 +497,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     ptx::tmem_ld16(tlane + j0 + 16, o1);
     ptx::tmem_ld16(tlane + kTile + j0, k0);
     ptx::tmem_ld16(tlane + kTile + j0 + 16, k1);
+    const float4 *gam4 = reinterpret_cast<const float4 *>(&ms.gam[j0]);
+    const float4 *bg4 = reinterpret_cast<const float4 *>(&ms.bg[j0]);
+    const float4 *bq4 = reinterpret_cast<const float4 *>(&ms.bq[j0]);
     ptx::tmem_wait_ld();
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      o0[j] *= ms.gam[j0 + j];
-      o1[j] *= ms.gam[j0 + 16 + j];
+    for (int j4 = 0; j4 < 4; ++j4) {
+      const float4 ga = gam4[j4], gb = gam4[4 + j4];
+      o0[4 * j4] *= ga.x; o0[4 * j4 + 1] *= ga.y; o0[4 * j4 + 2] *= ga.z; o0[4 * j4 + 3] *= ga.w;
+      o1[4 * j4] *= gb.x; o1[4 * j4 + 1] *= gb.y; o1[4 * j4 + 2] *= gb.z; o1[4 * j4 + 3] *= gb.w;
     }
     ptx::tmem_st16(tlane + j0, o0);
     ptx::tmem_st16(tlane + j0 + 16, o1);
@@ -505,33 +513,41 @@ __global__ void __launch_bounds__(kThreads, 2)
     const unsigned char *vt = sm + kOffV + (v >> 6) * kVHalf + (v & 7) * 2;
     const int vc = (v & 63) >> 3;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int ja = j0 + j, jb = j0 + 16 + j;
-      const float va = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(vt + ja * 128 + ((vc ^ (ja & 7)) << 4)));
-      const float vb = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(vt + jb * 128 + ((vc ^ (jb & 7)) << 4)));
-      k0[j] = ja < n_nodes ? tf32_rn(kGdn ? fmaf(-ms.bg[ja], k0[j], ms.bb[ja] * va) : va) : 0.f;
-      k1[j] = jb < n_nodes ? tf32_rn(kGdn ? fmaf(-ms.bg[jb], k1[j], ms.bb[jb] * vb) : vb) : 0.f;
+    for (int j4 = 0; j4 < 4; ++j4) {
+      const float4 ba = bq4[j4], bb = bq4[4 + j4], ca = bg4[j4], cb = bg4[4 + j4];
+      const float bja[4] = {ba.x, ba.y, ba.z, ba.w}, bjb[4] = {bb.x, bb.y, bb.z, bb.w};
+      const float cja[4] = {ca.x, ca.y, ca.z, ca.w}, cjb[4] = {cb.x, cb.y, cb.z, cb.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = 4 * j4 + e, ja = j0 + j, jb = j0 + 16 + j;
+        const float va = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(vt + ja * 128 + ((vc ^ (ja & 7)) << 4)));
+        const float vb = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(vt + jb * 128 + ((vc ^ (jb & 7)) << 4)));
+        k0[j] = ja < n_nodes ? tf32_rn(kGdn ? fmaf(-cja[e], k0[j], bja[e] * va) : va) : 0.f;
+        k1[j] = jb < n_nodes ? tf32_rn(kGdn ? fmaf(-cjb[e], k1[j], bjb[e] * vb) : vb) : 0.f;
+      }
     }
     ptx::tmem_st16(tlane + kColR + j0, k0);
     ptx::tmem_st16(tlane + kColR + j0 + 16, k1);
+    // the U columns start from zero
+#pragma unroll
+    for (int j = 0; j < 16; ++j) k0[j] = 0.f;
+    ptx::tmem_st16(tlane + kTile + j0, k0);
+    ptx::tmem_st16(tlane + kTile + j0 + 16, k0);
   }
   ptx::tmem_wait_st();
   ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
   __syncthreads();
 
-  // ---- 7. path-sum MMA: columns 0..63 += R^T . W^T, columns 64..127 = R^T . T^T (tf32) ---
+  // ---- 7. path-sum MMA: columns 0..127 += R^T . [W ; T]^T (tf32), i.e. o^T and U^T ------
   if (tid == kThreads - 1) {
     ptx::tc_fence_after();
-    constexpr uint32_t idesc = ptx::idesc_tf32_f32(128, 64);
+    constexpr uint32_t idesc = ptx::idesc_tf32_f32(128, 128);
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      const uint32_t kb = sbase + kOffA2 + (kk >> 2) * kAtom2 + (kk & 3) * 32;
-      const uint32_t ra = tmem + kColR + kk * 8;
-      ptx::mma_tf32_tmem_a(tmem, ra, ptx::smem_desc_sw128(kb, 1024), idesc, 1u);
-      ptx::mma_tf32_tmem_a(tmem + kTile, ra, ptx::smem_desc_sw128(kb + kTile * 128, 1024), idesc,
-                           kk > 0 ? 1u : 0u);
-    }
+    for (int kk = 0; kk < 8; ++kk)
+      ptx::mma_tf32_tmem_a(tmem, tmem + kColR + kk * 8,
+                           ptx::smem_desc_sw128(sbase + kOffA2 + (kk >> 2) * kAtom2 + (kk & 3) * 32, 1024),
+                           idesc, 1u);
     ptx::mma_commit(bar_sum);
   }
   if (!wait_all(ms, bar_sum, tid, a.ws, s)) {
