@@ -114,11 +114,11 @@ __device__ __forceinline__ float lds(const unsigned char *p, int off) {
 __device__ __forceinline__ void sts(unsigned char *p, int off, float x) {
   *reinterpret_cast<float *>(p + off) = x;
 }
-// fp32 -> nearest tf32 (ties away), kept in an fp32 container with the low 13 bits clear.
+// fp32 -> nearest tf32 (ties away from zero), kept in an fp32 container with the low 13
+// bits clear: half a unit of the 10-bit significand is added to the magnitude bits and the
+// 13 dropped bits are cleared (two integer operations; the tensor core ignores those bits).
 __device__ __forceinline__ float tf32_rn(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return __uint_as_float(r);
+  return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
 }
 // Streaming 16-byte load that stays where it is written: ahead of the tree-range check.
 __device__ __forceinline__ float4 ldg_first(const float4 *p) {
