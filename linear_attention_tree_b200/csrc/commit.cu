@@ -399,6 +399,11 @@ __global__ void __launch_bounds__(kSThreads, 1) commit_stream_kernel(CommitArgs 
   // a contiguous range of items per CTA: the heads of a sequence share its path row
   const int first = (int)((long long)blockIdx.x * n_items / gridDim.x);
   const int n = (int)((long long)(blockIdx.x + 1) * n_items / gridDim.x) - first;
+  // launched with programmatic stream serialisation: wait for the kernel before this one
+  // on the stream (U comes from it; S_new may alias S_root) before the first global access,
+  // and let the kernel after this one get its CTAs resident early
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(ptx::smem_addr(&sm.s_full[i]), 1);
@@ -529,8 +534,17 @@ cudaError_t launch_stream(const CommitArgs &a, cudaStream_t st) {
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = std::min(a.B * a.H, sms);
-  kern<<<grid, kSThreads, kStreamSmemBytes, st>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kSThreads);
+  cfg.dynamicSmemBytes = kStreamSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 cudaError_t launch_commit(const CommitArgs &a, int in_dtype, cudaStream_t st) {

@@ -232,6 +232,11 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H;
   const int s = blockIdx.x / H, h = blockIdx.x % H;
+  // launched with programmatic stream serialisation: the kernel before this one on the
+  // stream may still be finishing; wait for it (and its memory) before the first global
+  // read, and let the kernel after this one get its CTAs resident early
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // ---- 1. S_root loads, the tree's node range, q / k / v by TMA, tree inputs ----------
   // S_root as 16 float4 per thread: thread t owns 8-element k chunk (t & 15) of value rows
@@ -628,8 +633,17 @@ cudaError_t launch_tc_t(const VerifyArgs &a, cudaStream_t st) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  kern<<<a.B * a.H, kThreads, kSmemBytes, st>>>(mq, mk, mv, a, 2 * sms);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.B * a.H);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, a, 2 * sms);
 }
 
 }  // namespace
