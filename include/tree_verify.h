@@ -50,6 +50,14 @@
  * - workspace: device scratch of at least tv_workspace_size() bytes, 16-byte aligned,
  *   zero-filled by the caller before its first use; it holds the device status word.
  *   One workspace may serve many calls in stream order.
+ * - Stream order is kept.  The tensor-core verify kernel (dk = dv = 128) and the streaming
+ *   commit kernel are launched with programmatic stream serialisation.  Their CTAs may
+ *   become resident while the previous kernel on the stream drains, but they read and
+ *   write nothing before that kernel has completed.  They also signal programmatic
+ *   completion early.  A later kernel that the caller launches with programmatic
+ *   serialisation must therefore wait for its grid dependency (griddepcontrol.wait /
+ *   cudaGridDependencySynchronize) before it reads o, U or S_new.  Ordinary launches and
+ *   copies see the usual stream order.
  */
 #ifndef TREE_VERIFY_H
 #define TREE_VERIFY_H
