@@ -304,20 +304,42 @@ def run_b200(args, workloads):
     names = ["q", "k", "v", "log_a", "b", "parent", "node_offsets", "S_root", "accepted_path"]
     h2d = sum(host[0][n].numel() * host[0][n].element_size() for n in names)
     d2h = h_out[0].numel() * h_out[0].element_size() + h_S[0].numel() * 4
-    e2e_steps = max(3, min(args.steps, 20))
+    e2e_steps = max(3, min(args.steps, 50))
+
+    # pipelined over the three buffer sets: inputs go up on one stream, the step runs on
+    # the launching stream, results come down on a third, so that copies in both
+    # directions overlap other steps' kernels
+    copy_in, copy_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    in_ready = [torch.cuda.Event() for _ in range(N_SETS)]
+    done = [torch.cuda.Event() for _ in range(N_SETS)]
+    out_read = [torch.cuda.Event() for _ in range(N_SETS)]
+    used = [False] * N_SETS
 
     def e2e_step(i):
-        h, d = host[i % N_SETS], sets[i % N_SETS]
-        o, U, S_new = outs[i % N_SETS]
-        for n in names:
-            d[n].copy_(h[n], non_blocking=True)
+        slot = i % N_SETS
+        h, d = host[slot], sets[slot]
+        o, U, S_new = outs[slot]
+        if used[slot]:
+            copy_in.wait_event(done[slot])          # the last step on this slot has read it
+        with torch.cuda.stream(copy_in):
+            for n in names:
+                d[n].copy_(h[n], non_blocking=True)
+            in_ready[slot].record(copy_in)
+        stream.wait_event(in_ready[slot])
+        if used[slot]:
+            stream.wait_event(out_read[slot])       # its previous results have been copied out
         L.tree_verify(d["q"], d["k"], d["v"], d["log_a"], d["b"], d["parent"],
                       d["node_offsets"], d["S_root"], max_nodes=w0.max_nodes, out=o, U=U,
                       workspace=ws, kernel=args.kernel)
         L.tree_commit(U, d["k"], d["log_a"], d["S_root"], d["node_offsets"],
                       d["accepted_path"], max_nodes=w0.max_nodes, S_new=S_new, workspace=ws)
-        h_out[i % N_SETS].copy_(o, non_blocking=True)
-        h_S[i % N_SETS].copy_(S_new, non_blocking=True)
+        done[slot].record(stream)
+        copy_out.wait_event(done[slot])
+        with torch.cuda.stream(copy_out):
+            h_out[slot].copy_(o, non_blocking=True)
+            h_S[slot].copy_(S_new, non_blocking=True)
+            out_read[slot].record(copy_out)
+        used[slot] = True
 
     for i in range(3):
         e2e_step(i)
@@ -325,8 +347,12 @@ def run_b200(args, workloads):
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    copy_in.wait_event(e0)
+    copy_out.wait_event(e0)
     for i in range(e2e_steps):
         e2e_step(i)
+    stream.wait_stream(copy_out)
+    stream.wait_stream(copy_in)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
