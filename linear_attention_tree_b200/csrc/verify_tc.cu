@@ -25,9 +25,9 @@
 //      128-byte swizzled layout the MMA reads.
 //   2. Gram MMA (tcgen05 kind::f16, 128 x 64 x 128): [Q ; K] . K^T into columns 128..191,
 //      as soon as q and k have landed; meanwhile the tree is walked.
-//   3-4. Gram entries by path position, then the T and W row recursions -- none of which
-//      needs S_root, so they run while S_root is still arriving; then S_root -> bf16.
-//   5. state MMA (kind::f16, 128 x 128 x 128): S_root . [Q ; K]^T into columns 0..127.
+//   3. Gram entries by path position (they need no S_root); S_root -> bf16.
+//   4-5. state MMA (kind::f16, 128 x 128 x 128): S_root . [Q ; K]^T into columns 0..127,
+//      while warps 0-3 run the T and W row recursions.
 //   6. per value lane: columns 0..63 scaled by gamma_n; R^T[v][j] = b_j v_j[v] -
 //      b_j gamma_j (S_root k_j)[v] into columns 192..255 (tf32); [W ; T] written as the
 //      shared-memory operand.
@@ -390,17 +390,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         if ((bits >> j) & 1u) pos_major[pos++][gn] = scale * g[j];
     }
   }
-  __syncthreads();
-
-  // ---- 4. T and W rows (shallow trees, warps 0-3) while S_root arrives; S_root -> bf16 --
-  if (fast && tid < 2 * kTile) {
-    const int m = tid & (kTile - 1);
-    if (m < n_nodes) {
-      const int d = ms.dep[m];
-      if (tid < kTile) row_coefficients<true, kGdn>(ms, paths, m, d);
-      else row_coefficients<false, kGdn>(ms, paths, m, d);
-    }
-  }
+  // S_root -> bf16 operand rows (all threads; the loads have long arrived by now)
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int v = (tid >> 4) + 16 * j;
@@ -420,12 +410,23 @@ __global__ void __launch_bounds__(kThreads, 2)
   ptx::tc_fence_before();
   __syncthreads();
 
-  // ---- 5. state MMA: columns 0..127 = S_root . [Q ; K]^T ------------------------------------
+  // ---- 4. state MMA: columns 0..127 = S_root . [Q ; K]^T; meanwhile warps 0-3 run the T
+  // and W row recursions of shallow trees -------------------------------------------------
   if (tid == kThreads - 1) {
     ptx::tc_fence_after();
     mma_chain_bf16(sbase + kOffS, sbase + kOffQK, tmem, ptx::idesc_bf16_f32(128, 128));
     ptx::mma_commit(bar_state);
   }
+  if (fast && tid < 2 * kTile) {
+    const int m = tid & (kTile - 1);
+    if (m < n_nodes) {
+      const int d = ms.dep[m];
+      if (tid < kTile) row_coefficients<true, kGdn>(ms, paths, m, d);
+      else row_coefficients<false, kGdn>(ms, paths, m, d);
+    }
+  }
+
+  // ---- 5. the state product has landed (the barrier also publishes the T and W rows) -----
   if (!wait_all(ms, bar_state, tid, a.ws, s)) {
     release_tmem(warp, tmem);
     return;
