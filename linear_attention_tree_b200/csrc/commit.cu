@@ -399,10 +399,10 @@ __global__ void __launch_bounds__(kSThreads, 1) commit_stream_kernel(CommitArgs 
   // a contiguous range of items per CTA: the heads of a sequence share its path row
   const int first = (int)((long long)blockIdx.x * n_items / gridDim.x);
   const int n = (int)((long long)(blockIdx.x + 1) * n_items / gridDim.x) - first;
-  // launched with programmatic stream serialisation: wait for the kernel before this one
-  // on the stream (U comes from it; S_new may alias S_root) before the first global access,
-  // and let the kernel after this one get its CTAs resident early
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // Launched with programmatic stream serialisation.  The mover's first two S_root copies
+  // go out before the grid dependency is waited for (S_root is only read by the verify
+  // kernel that precedes this one); every other global access -- U and the path inputs,
+  // and the stores that may alias S_root -- waits for the previous kernel to complete.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -418,12 +418,14 @@ __global__ void __launch_bounds__(kSThreads, 1) commit_stream_kernel(CommitArgs 
   }
   __syncthreads();
 
+  if (warp != kSMoverWarp) asm volatile("griddepcontrol.wait;" ::: "memory");
   if (warp == kSMoverWarp) {
     if (lane == 0) {
       // item li goes into stage li & 1 once the compute warps have read item li - 2 from it
       int loaded = 0;
       for (int li = 0; li < n; ++li) {
         const int st = li & 1;
+        if (li == 2) asm volatile("griddepcontrol.wait;" ::: "memory");
         if (li >= 2 &&
             !stream_wait(sm, ptx::smem_addr(&sm.s_empty[st]), ((li - 2) >> 1) & 1, a.ws, first / a.H))
           break;
@@ -433,6 +435,7 @@ __global__ void __launch_bounds__(kSThreads, 1) commit_stream_kernel(CommitArgs 
                        kStateBytes, full);
         loaded = li + 1;
       }
+      if (n < 2) asm volatile("griddepcontrol.wait;" ::: "memory");
       if (*reinterpret_cast<volatile int *>(&sm.fail))
         // after a time-out: let the state copies still in flight land before the CTA's
         // shared memory is released (bounded)
