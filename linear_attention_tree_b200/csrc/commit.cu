@@ -7,17 +7,17 @@
 //
 // One CTA per (sequence, head, slice of kRows state rows).  The kernel is HBM bound (one
 // read and one write of the state), so everything that depends on the path is kept to
-// two rounds of dependent global loads, overlapped with the state loads:
-//   round 0: the state slice (registers), node_offsets, the accepted_path row (warp 0,
+// two sets of dependent global loads, overlapped with the state loads:
+//   first loads: the state slice (registers), node_offsets, the accepted_path row (warp 0,
 //            checked with one ballot per 32 entries);
-//   round 1: parent and log_a of the path nodes and their u and k rows, all at once.
+//   second loads: parent and log_a of the path nodes and their u and k rows, all at once.
 // Then one thread forms the fp32 prefix sums c_j (root first, the order the verify
 // kernels use for cl), the u rows are scaled, and S_new streams out with 128-bit stores.
 //
 // For dk = dv = 128 a streaming form replaces it: persistent CTAs (one per SM) walk a
 // contiguous range of (sequence, head) states.  Each 64 KiB state arrives by bulk copy into
 // a two-stage shared-memory ring one item ahead, and a loader warp gathers the next item's
-// path (the two dependent rounds above) while sixteen warps rebuild and store the current
+// path (the two dependent load sets above) while sixteen warps rebuild and store the current
 // one, so the state stream never waits on the path gather.
 #include <algorithm>
 #include <cstddef>
@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(CommitArgs a) {
   const int rows = min(kRows, dv - r0);
   const Tk *k = static_cast<const Tk *>(a.k);
 
-  // ---- round 0 ---------------------------------------------------------------------
+  // ---- first loads -----------------------------------------------------------------
   const size_t base = (((size_t)s * H + h) * dv + r0) * dk;
   const float4 *Sg = reinterpret_cast<const float4 *>(a.S_root + base);
   const int nvec = rows * dk / 4;
@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(CommitArgs a) {
   }
   const int m = sm.m, lo = sm.lo;
 
-  // ---- round 1: parent / log_a of the path, the first chunk of u and k rows ----------
+  // ---- second loads: parent / log_a of the path, the first chunk of u and k rows -----
   int chain_bad = 0;
   for (int t = tid; t < m; t += kThreads) {
     const int p = sm.prow[t];
