@@ -324,7 +324,7 @@ __device__ void gather_path(const CommitArgs &a, int it, PathBuf &pb, const Path
   gather_rows<Tk>(a, it, pb, m, lo, lane);
 }
 
-// Gatherer warp, second round: log_a and the parent chain of the m path entries (row already
+// Gatherer warp, second load set: log_a and the parent chain of the m path entries (row already
 // in pb.prow), decay weights, and the u and k rows of the first kPathRows entries.
 template <typename Tk>
 __device__ void gather_rows(const CommitArgs &a, int it, PathBuf &pb, int m, int lo, int lane) {
