@@ -109,3 +109,12 @@ def test_product_path_has_no_cpu_fallback():
         if fn.endswith(".py"):
             assert "import oracle" not in open(os.path.join(pkg, fn)).read()
             assert "from oracle" not in open(os.path.join(pkg, fn)).read()
+
+
+def test_workspace_is_constant_size():
+    """The workspace holds only the status word: its size does not grow with the number of
+    nodes, heads or the state size (there are no per-node state snapshots anywhere)."""
+    small = L.workspace_size(L.make_problem(1, 1, 16, 16, 6, 6, 3))
+    big = L.workspace_size(L.make_problem(128, 32, 128, 128, 3072, 48, 7))
+    wide = L.workspace_size(L.make_problem(8, 32, 128, 128, 2048, 256, 11))
+    assert 0 < small == big == wide <= 4096

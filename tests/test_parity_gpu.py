@@ -87,7 +87,8 @@ def test_full_size_sampled_simt(idx):
     _sampled_check(W.config(idx), kernel="simt", n_nodes=60, n_states=8, seed=1)
 
 
-@pytest.mark.parametrize("idx,seed", [(3, 1), (3, 2), (4, 1)])
+@pytest.mark.parametrize("idx,seed", [(2, 1), (2, 2), (2, 3), (3, 1), (3, 2), (3, 3), (4, 1),
+                                      (4, 2), (5, 1)])
 def test_extra_seeds(idx, seed):
     _sampled_check(W.config(idx, seed=seed), n_nodes=60, n_states=8, seed=seed)
 
@@ -98,6 +99,14 @@ def _ragged(seed, counts, max_depth=8, fmax=4):
         par, _ = W.frontier_tree(seed * 100 + i, c, max_depth, fmax) if c else ([], None)
         pars.append(par)
     return pars
+
+
+def test_node_counts_past_the_tensor_core_tile():
+    """65 and 255 nodes per tree (the CUDA-core kernel, picked automatically), with a 1-node
+    tree beside them, compared in full."""
+    w = W.synthetic(_ragged(9, [65, 1, 255], max_depth=10, fmax=6), H=2, dk=128, dv=128,
+                    seed=321, name="ragged-wide")
+    _full_check(w, "auto")
 
 
 @pytest.mark.parametrize("kernel", ["tc", "simt"])
