@@ -50,17 +50,17 @@
  * - workspace: device scratch of at least tv_workspace_size() bytes, 16-byte aligned,
  *   zero-filled by the caller before its first use; it holds the device status word.
  *   One workspace may serve many calls in stream order.
- * - Stream order is kept.  The tensor-core verify kernel (dk = dv = 128) and the streaming
- *   commit kernel are launched with programmatic stream serialisation.  Their CTAs may
- *   become resident while the previous kernel on the stream drains.  Apart from one
- *   exception, they read and write nothing before that kernel has completed.  The
+ * - Stream order is kept.  The tensor-core verify kernel (dk = dv = 128) and the
+ *   streaming commit kernel are launched with programmatic stream serialisation.  Their
+ *   CTAs may become resident while the previous kernel on the stream drains.  Apart from
+ *   one exception, they read and write nothing before that kernel has completed.  The
  *   exception: tv_tree_commit may start copying its first S_root blocks as soon as that
- *   kernel has signalled programmatic completion.  tv_tree_verify never writes S_root, but
- *   a caller's own kernel that signals early must not write S_root either.  Both kernels
- *   also signal programmatic completion early.  A later kernel that the caller launches with programmatic
- *   serialisation must therefore wait for its grid dependency (griddepcontrol.wait /
- *   cudaGridDependencySynchronize) before it reads o, U or S_new.  Ordinary launches and
- *   copies see the usual stream order.
+ *   kernel has signalled programmatic completion.  tv_tree_verify never writes S_root,
+ *   but a caller's own kernel that signals early must not write S_root either.  Both
+ *   kernels also signal programmatic completion early.  A later kernel that the caller
+ *   launches with programmatic serialisation must therefore wait for its grid dependency
+ *   (griddepcontrol.wait / cudaGridDependencySynchronize) before it reads o, U or S_new.
+ *   Ordinary launches and copies see the usual stream order.
  */
 #ifndef TREE_VERIFY_H
 #define TREE_VERIFY_H
@@ -192,6 +192,15 @@ TV_API tv_status tv_tree_verify_noalloc(const tv_problem *p, const void *q, cons
                                         const int32_t *parent, const int32_t *node_offsets,
                                         const float *S_root, void *out, float *U,
                                         void **scratch_out, tv_stream_t stream);
+
+/* Diagnostic, with no counterpart on the pages: enqueue one small kernel whose bounded
+ * wait on an mbarrier phase that never completes runs out.  It then records
+ * TV_ERR_TIMEOUT in `workspace`, as a verify or commit CTA does after a wait that does not
+ * complete.  This is for testing the time-out path: nothing faults or hangs, and the
+ * context stays usable.  A NULL, misaligned or too small workspace returns
+ * TV_ERR_INVALID_ARG. */
+TV_API tv_status tv_selftest_timeout(void *workspace, size_t workspace_bytes,
+                                     tv_stream_t stream);
 
 /* Synchronise `stream`, return the first device-side error recorded in `workspace` since
  * the last call (TV_OK if none) and clear it.  Not for the hot path. */

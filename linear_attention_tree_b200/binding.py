@@ -11,6 +11,7 @@ Python name  -> C entry point
   tree_meta       tv_tree_meta
   workspace_size  tv_workspace_size
   get_status      tv_get_status
+  selftest_timeout tv_selftest_timeout
 """
 from __future__ import annotations
 
@@ -29,7 +30,8 @@ MODE = {"gdn": 0, "scalar": 1}
 DTYPE = {torch.float32: 0, torch.bfloat16: 1}
 KERNEL = {"auto": 0, "tc": 1, "simt": 2}
 EXPORTS = ("tv_workspace_size", "tv_tree_verify", "tv_tree_commit", "tv_tree_meta",
-           "tv_get_status", "tv_status_string", "tv_last_cuda_error", "tv_version")
+           "tv_get_status", "tv_status_string", "tv_last_cuda_error", "tv_version",
+           "tv_selftest_timeout")
 
 
 class TreeVerifyError(RuntimeError):
@@ -70,6 +72,8 @@ def lib() -> ctypes.CDLL:
         L.tv_tree_meta.restype = ctypes.c_int
         L.tv_get_status.argtypes = [vp, vp]
         L.tv_get_status.restype = ctypes.c_int
+        L.tv_selftest_timeout.argtypes = [vp, ctypes.c_size_t, vp]
+        L.tv_selftest_timeout.restype = ctypes.c_int
         L.tv_status_string.argtypes = [ctypes.c_int]
         L.tv_status_string.restype = ctypes.c_char_p
         L.tv_last_cuda_error.argtypes = []
@@ -229,6 +233,13 @@ def tree_meta(parent, node_offsets, log_a, *, max_nodes: int, workspace=None, st
                             _stream(stream))
     _check(st, "tv_tree_meta")
     return depth, anc, cumlog
+
+
+def selftest_timeout(workspace: torch.Tensor, stream=None) -> None:
+    """Enqueue the library's time-out diagnostic: a bounded wait that runs out records
+    TV_ERR_TIMEOUT in ``workspace`` (read it with `get_status`)."""
+    _check(lib().tv_selftest_timeout(_ptr(workspace, "workspace", torch.uint8),
+                                     workspace.numel(), _stream(stream)), "selftest_timeout")
 
 
 def get_status(workspace: torch.Tensor, stream=None) -> int:

@@ -156,6 +156,13 @@ tv_status tv_tree_meta(const tv_problem *p, const int32_t *parent,
   return from_cuda(launch_meta(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+tv_status tv_selftest_timeout(void *workspace, size_t workspace_bytes, tv_stream_t stream) {
+  if (!ptr_ok(workspace) || workspace_bytes < kWorkspaceBytes) return TV_ERR_INVALID_ARG;
+  // a short poll budget: the point is the path taken when a wait runs out, not its length
+  return from_cuda(launch_timeout_probe(static_cast<int *>(workspace), 4096,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
 tv_status tv_get_status(void *workspace, tv_stream_t stream) {
   if (!ptr_ok(workspace)) return TV_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -63,6 +63,7 @@ struct MetaArgs {
 };
 
 // Launchers (host side); each returns cudaSuccess or the launch error.
+cudaError_t launch_timeout_probe(int *ws, uint32_t polls, cudaStream_t st);
 cudaError_t launch_verify_simt(const VerifyArgs &a, int mode, int in_dtype, int out_dtype,
                                cudaStream_t st);
 int verify_tc_max_nodes();

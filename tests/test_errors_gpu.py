@@ -107,3 +107,17 @@ def test_unsupported_kernel_raises():
     ws = L.new_workspace(L.make_problem(w.B, w.H, w.dk, w.dv, w.T, w.max_nodes))
     with pytest.raises(L.TreeVerifyError):
         _verify(w, d, ws, kernel="tc")
+
+
+def test_wait_that_runs_out_is_reported_and_the_context_survives():
+    """A bounded mbarrier wait that never completes (the library's diagnostic kernel) ends
+    with TV_ERR_TIMEOUT in the status word instead of a hang; the next call is correct."""
+    w = W.config(2)
+    ws = L.new_workspace(L.make_problem(w.B, w.H, w.dk, w.dv, w.T, w.max_nodes, w.max_path))
+    L.binding.selftest_timeout(ws)
+    assert L.get_status(ws) == L.binding.TV_ERR_TIMEOUT
+    assert L.get_status(ws) == 0                      # read once, then cleared
+    res, _ = run(w)
+    o, U = O.tree_verify(w)
+    assert_close(res["o"], o, TOL["bf16"], "o after a time-out")
+    assert_close(res["U"], U, TOL["bf16"], "U after a time-out")
