@@ -118,3 +118,10 @@ def test_workspace_is_constant_size():
     big = L.workspace_size(L.make_problem(128, 32, 128, 128, 3072, 48, 7))
     wide = L.workspace_size(L.make_problem(8, 32, 128, 128, 2048, 256, 11))
     assert 0 < small == big == wide <= 4096
+
+
+def test_selftest_rejects_bad_workspace_before_launching():
+    f = L.lib().tv_selftest_timeout
+    assert f(None, 256, None) == binding.TV_ERR_INVALID_ARG
+    assert f(ctypes.c_void_p(0x10004), 256, None) == binding.TV_ERR_INVALID_ARG
+    assert f(ctypes.c_void_p(0x10000), 8, None) == binding.TV_ERR_INVALID_ARG
