@@ -52,12 +52,11 @@
  *   One workspace may serve many calls in stream order.
  * - Stream order is kept.  The tensor-core verify kernel (dk = dv = 128) and the
  *   streaming commit kernel are launched with programmatic stream serialisation.  Their
- *   CTAs may become resident while the previous kernel on the stream drains.  Apart from
- *   one exception, they read and write nothing before that kernel has completed.  The
- *   exception: tv_tree_commit may start copying its first S_root blocks as soon as that
- *   kernel has signalled programmatic completion.  tv_tree_verify never writes S_root,
- *   but a caller's own kernel that signals early must not write S_root either.  Both
- *   kernels also signal programmatic completion early.  A later kernel that the caller
+ *   CTAs may become resident while the previous kernel on the stream drains, and may ask
+ *   L2 to prefetch their first inputs then, but they load and store nothing before that
+ *   kernel has completed; any sequence of library calls on one stream (commit after
+ *   commit on chained or in-place states included) therefore sees plain stream order.
+ *   Both kernels signal programmatic completion early.  A later kernel that the caller
  *   launches with programmatic serialisation must therefore wait for its grid dependency
  *   (griddepcontrol.wait / cudaGridDependencySynchronize) before it reads o, U or S_new.
  *   Ordinary launches and copies see the usual stream order.

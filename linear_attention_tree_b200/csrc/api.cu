@@ -48,6 +48,10 @@ tv_status from_cuda(cudaError_t e) {
 
 }  // namespace
 
+namespace tv {
+tv_status record_cuda_error(cudaError_t e) { return from_cuda(e); }
+}  // namespace tv
+
 extern "C" {
 
 int32_t tv_version(void) { return (1 << 16) | 0; }

@@ -399,10 +399,11 @@ __global__ void __launch_bounds__(kSThreads, 1) commit_stream_kernel(CommitArgs 
   // a contiguous range of items per CTA: the heads of a sequence share its path row
   const int first = (int)((long long)blockIdx.x * n_items / gridDim.x);
   const int n = (int)((long long)(blockIdx.x + 1) * n_items / gridDim.x) - first;
-  // Launched with programmatic stream serialisation.  The mover's first two S_root copies
-  // go out before the grid dependency is waited for (S_root is only read by the verify
-  // kernel that precedes this one); every other global access -- U and the path inputs,
-  // and the stores that may alias S_root -- waits for the previous kernel to complete.
+  // Launched with programmatic stream serialisation.  Before the grid dependency resolves
+  // the mover only asks L2 to prefetch its first two S_root blocks: a prefetch moves no
+  // data into this CTA, and a write by the previous kernel to the same lines lands in L2
+  // after it, so this is correct whatever that kernel writes (another commit's S_new
+  // included).  Every load and store waits for the previous kernel to complete.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -418,14 +419,16 @@ __global__ void __launch_bounds__(kSThreads, 1) commit_stream_kernel(CommitArgs 
   }
   __syncthreads();
 
-  if (warp != kSMoverWarp) asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (warp == kSMoverWarp && lane == 0)
+    for (int li = 0; li < n && li < 2; ++li)
+      ptx::prefetch_l2(a.S_root + (size_t)(first + li) * 128 * 128, kStateBytes);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (warp == kSMoverWarp) {
     if (lane == 0) {
       // item li goes into stage li & 1 once the compute warps have read item li - 2 from it
       int loaded = 0;
       for (int li = 0; li < n; ++li) {
         const int st = li & 1;
-        if (li == 2) asm volatile("griddepcontrol.wait;" ::: "memory");
         if (li >= 2 &&
             !stream_wait(sm, ptx::smem_addr(&sm.s_empty[st]), ((li - 2) >> 1) & 1, a.ws, first / a.H))
           break;
@@ -435,7 +438,6 @@ __global__ void __launch_bounds__(kSThreads, 1) commit_stream_kernel(CommitArgs 
                        kStateBytes, full);
         loaded = li + 1;
       }
-      if (n < 2) asm volatile("griddepcontrol.wait;" ::: "memory");
       if (*reinterpret_cast<volatile int *>(&sm.fail))
         // after a time-out: let the state copies still in flight land before the CTA's
         // shared memory is released (bounded)

@@ -56,7 +56,8 @@ extern "C" tv_status tv_tree_verify_noalloc(const tv_problem *p, const void *q, 
                           0, stream);
   if (need > kStaticScratchBytes) return TV_ERR_UNSUPPORTED;
   void *scratch = nullptr;
-  if (scratch_for_current_device(&scratch) != cudaSuccess) return TV_ERR_CUDA;
+  const cudaError_t e = scratch_for_current_device(&scratch);
+  if (e != cudaSuccess) return tv::record_cuda_error(e);   // readable via tv_last_cuda_error
   if (scratch_out) *scratch_out = scratch;
   return tv_tree_verify(p, q, k, v, log_a, b, parent, node_offsets, S_root, out, U, scratch,
                         kStaticScratchBytes, stream);

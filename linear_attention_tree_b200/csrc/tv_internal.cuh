@@ -62,6 +62,10 @@ struct MetaArgs {
   int B, H, T, max_nodes, anc_words;
 };
 
+// Record a failed CUDA call for tv_last_cuda_error on the calling host thread and return
+// TV_ERR_CUDA (TV_OK for cudaSuccess).  Every entry point reports CUDA failures this way.
+tv_status record_cuda_error(cudaError_t e);
+
 // Launchers (host side); each returns cudaSuccess or the launch error.
 cudaError_t launch_timeout_probe(int *ws, uint32_t polls, cudaStream_t st);
 cudaError_t launch_verify_simt(const VerifyArgs &a, int mode, int in_dtype, int out_dtype,

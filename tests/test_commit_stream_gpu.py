@@ -77,3 +77,43 @@ def test_in_place_long_paths():
     L.tree_commit(U, d["k"], d["log_a"], S, d["node_offsets"], d["accepted_path"],
                   max_nodes=w.max_nodes, S_new=S)
     torch.testing.assert_close(S, S_new, rtol=0, atol=0)
+
+
+@pytest.mark.parametrize("in_place", [False, True])
+def test_two_commits_back_to_back_on_chained_states(in_place):
+    """commit -> commit on one stream, the second reading the first one's S_new (a new
+    buffer, or S_root itself in place), with nothing between them.  Scalar decay makes
+    U = V valid for any root state, so the second commit's pseudo-values need no verify
+    on the intermediate state; the oracle walks path A from S_root, then path B."""
+    pars = [W.frontier_tree(600 + s, 40, 8, 3)[0] for s in range(40)]
+    rng = np.random.default_rng(61)
+    paths_a, paths_b = [], []
+    for p in pars:
+        d = W.depths_of(p)
+        paths_a.append(O.path_to(p, int(rng.integers(0, len(p)))))
+        paths_b.append(O.path_to(p, int(np.argmax(d))))
+    w = W.synthetic(pars, H=8, dk=128, dv=128, seed=61, mode="scalar", paths=paths_a,
+                    log_a_mean=-3.0)
+    d = to_device(w)
+    U = d["v"].float().contiguous()                    # scalar decay: u_n = v_n
+    width = max(len(p) for p in paths_a + paths_b)
+    pad = lambda ps: torch.tensor([p + [-1] * (width - len(p)) for p in ps],
+                                  dtype=torch.int32, device="cuda")
+    path_a, path_b = pad(paths_a), pad(paths_b)
+    ws = L.new_workspace(L.make_problem(w.B, w.H, 128, 128, w.T, w.max_nodes, width))
+    S0 = d["S_root"].clone()
+    mid = S0 if in_place else torch.empty_like(S0)
+    L.tree_commit(U, d["k"], d["log_a"], S0, d["node_offsets"], path_a,
+                  max_nodes=w.max_nodes, parent=d["parent"], S_new=mid, workspace=ws)
+    end = mid if in_place else torch.empty_like(S0)
+    L.tree_commit(U, d["k"], d["log_a"], mid, d["node_offsets"], path_b,
+                  max_nodes=w.max_nodes, parent=d["parent"], S_new=end, workspace=ws)
+    assert L.get_status(ws) == 0
+    got = end.cpu().numpy().astype(np.float64)
+    want = np.empty_like(got)
+    for s in range(w.B):
+        for h in range(w.H):
+            q, k, v, la, b, S, parent = O._head(w, s, h)
+            S = O.walk(S, paths_a[s], k, v, la, b, "scalar")[0]
+            want[s, h] = O.walk(S, paths_b[s], k, v, la, b, "scalar")[0]
+    assert_close(got, want, TOL["bf16"], "S_new after two chained commits")

@@ -422,6 +422,71 @@ def test_meta_worked_example():
     np.testing.assert_allclose(cl[:, 0], np.array(depth) * np.float64(w.log_a[0, 0]), rtol=1e-15)
 
 
+def pin_meta_varied_decay():
+    """Cumulative log-decay with a different log_a on every node.
+
+    (a) Hand-summed values on a 6-node tree (root children 0 and 2, chain 0 -> 1 -> 3,
+    2 -> 4, 3 -> 5), one head: cl_n is the sum of log_a over the root -> n path, n
+    included (the worked example's depth-2 node carries lambda^2: one factor per path
+    token).  (b) With k = 0 in scalar mode the walk only decays, so the walked state is
+    exp(cl_n) S_root: the metadata must agree with the recurrence on random trees with
+    random per-node, per-head decays.
+    """
+    parent = [-1, 0, -1, 1, 2, 3]
+    log_a = np.array([[-0.5], [-0.25], [-2.0], [-0.125], [-1.0], [-0.0625]])
+    depth, anc, cl = O.tree_meta(parent, log_a)
+    assert list(depth) == [1, 2, 1, 3, 2, 4]
+    assert anc == [[], [0], [], [0, 1], [2], [0, 1, 3]]
+    want = np.array([-0.5, -0.75, -2.0, -0.875, -3.0, -0.9375])
+    np.testing.assert_array_equal(cl[:, 0], want)       # exact: dyadic values
+    rng = np.random.default_rng(43)
+    for trial in range(3):
+        par = W.uniform_parent_tree(rng, 12, 6)
+        w = W.synthetic([par], H=3, dk=4, dv=3, seed=43 + trial, mode="scalar", in_dtype="f32")
+        w.log_a = rng.uniform(-1.5, -0.01, size=w.log_a.shape).astype(np.float32)
+        w.k[:] = 0.0
+        _, _, cl = O.tree_meta(w.seq_parent(0), w.log_a)
+        for h in range(w.H):
+            S = O.node_states(w, 0, h)
+            ratio = S / w.S_root[0, h].astype(np.float64)
+            np.testing.assert_allclose(ratio, np.exp(cl[:, h])[:, None, None] *
+                                       np.ones_like(ratio), rtol=1e-13)
+
+
+def test_meta_varied_decay():
+    pin_meta_varied_decay()
+
+
+def _mut_meta_depth_times_own(parent, log_a):
+    depth, anc, _ = _orig_tree_meta(parent, log_a)
+    return depth, anc, depth[:, None] * np.asarray(log_a, dtype=np.float64)
+
+
+def _mut_meta_parent_excluded(parent, log_a):
+    depth, anc, cl = _orig_tree_meta(parent, log_a)
+    return depth, anc, cl - np.asarray(log_a, dtype=np.float64)
+
+
+def _mut_meta_first_node_decay(parent, log_a):
+    depth, anc, _ = _orig_tree_meta(parent, log_a)
+    la = np.asarray(log_a, dtype=np.float64)
+    return depth, anc, np.array([la[([*a, n])[0]] * d for n, (a, d) in
+                                 enumerate(zip(anc, depth))])
+
+
+_orig_tree_meta = O.tree_meta
+
+
+@pytest.mark.parametrize("mutant", [_mut_meta_depth_times_own, _mut_meta_parent_excluded,
+                                    _mut_meta_first_node_decay],
+                         ids=lambda m: m.__name__)
+def test_meta_pin_catches_planted_mistakes(monkeypatch, mutant):
+    """A per-node mix-up of log_a along the path fails the varied-decay pin."""
+    monkeypatch.setattr(O, "tree_meta", mutant)
+    with pytest.raises(AssertionError):
+        pin_meta_varied_decay()
+
+
 def test_commit_empty_path_is_root_and_matches_node_states():
     rng = np.random.default_rng(41)
     par = W.uniform_parent_tree(rng, 10, 4)

@@ -1,10 +1,11 @@
 """Parity of the CUDA path with the float64 oracle, element by element.
 
 Bars: max|err| <= 1e-4 * RMS(oracle tensor) for fp32 inputs, <= 2e-2 * RMS for bf16
-inputs, separately for o, U and S_new.  Small problems are compared in full; the five
-named workloads at full size are compared in full where the oracle is quick (1, 2) and on
-seeded samples of (node, head) outputs and (sequence, head) states otherwise, in the same
-launch configuration the benchmark times.
+inputs, separately for o, U and S_new.  Every one of the five named workloads is compared
+in full, every node, head and state: 1 and 2 directly, 3-5 against the oracle spread over
+the host's cores (``tests/_oracle_pool.py``), with both kernels and in the launch
+configuration the benchmark times.  Smaller trees of every shape class (ragged, empty,
+deep branched, combs, chains) are compared in full as well.
 """
 import numpy as np
 import pytest
@@ -12,6 +13,15 @@ import pytest
 from linear_attention_tree_b200 import workloads as W
 from oracle import oracle as O
 from tests._gpu_util import TOL, assert_close, run
+from tests._oracle_pool import oracle_config
+
+_FULL = {}
+
+
+def _oracle_full(idx):
+    if idx not in _FULL:
+        _FULL[idx] = oracle_config(idx)
+    return _FULL[idx]
 
 pytestmark = pytest.mark.gpu
 
@@ -60,6 +70,19 @@ def test_config1_worked_example(kernel):
 @pytest.mark.parametrize("kernel", ["auto", "simt", "tc"])
 def test_config2(kernel):
     _full_check(W.config(2), kernel)
+
+
+@pytest.mark.parametrize("kernel", ["auto", "simt"])
+@pytest.mark.parametrize("idx", [3, 4, 5])
+def test_full_size_every_output(idx, kernel):
+    """Whole workloads 3-5 against the float64 oracle: every o and U row of every node and
+    head, every accepted state."""
+    w, o, U, S_new = _oracle_full(idx)
+    res, _ = run(w, kernel=kernel)
+    tol = TOL[w.in_dtype]
+    assert_close(res["o"], o, tol, f"o config {idx} {kernel}")
+    assert_close(res["U"], U, tol, f"U config {idx} {kernel}")
+    assert_close(res["S_new"], S_new, tol, f"S_new config {idx} {kernel}")
 
 
 @pytest.mark.parametrize("idx", [3, 4, 5])
@@ -157,3 +180,47 @@ def test_deep_chain_256():
     w = W.synthetic([[i - 1 for i in range(256)]], H=1, dk=64, dv=64, seed=8, in_dtype="f32",
                     log_a_mean=-5.0, s_std=0.05)
     _full_check(w, "auto")
+
+
+def _comb(spine):
+    """A spine of ``spine`` nodes with one leaf hanging off every spine node, interleaved in
+    topological order: node 2i is spine node i, node 2i+1 its leaf."""
+    par = []
+    for i in range(spine):
+        par.append(2 * (i - 1) if i else -1)
+        par.append(2 * i)
+    return par
+
+
+def _deep_branched_trees():
+    return {
+        # random frontier growth allowed to reach depth 40 with branching <= 2
+        "frontier64_d40": [W.frontier_tree(2024, 64, 40, 2)[0]],
+        # depth 33 comb: every node has a sparse ancestor set off the spine
+        "comb64": [_comb(32)],
+        # just past the register-recursion depth, next to shallow and tiny trees
+        "mixed_d9": [W.frontier_tree(77, 64, 9, 3)[0], W.frontier_tree(78, 40, 12, 2)[0],
+                     [-1], _comb(5)],
+        # two long branches that share a stem of 4 nodes
+        "fork": [[-1, 0, 1, 2] + [3] + list(range(4, 32)) + [3] + list(range(33, 62))],
+    }
+
+
+@pytest.mark.parametrize("kernel", ["tc", "simt"])
+@pytest.mark.parametrize("name", sorted(_deep_branched_trees()))
+def test_deep_branched_trees(name, kernel):
+    """Branched trees deeper than the tensor-core kernel's register recursion (depth > 8),
+    whose nodes have sparse ancestor sets, compared in full with paths to the deepest
+    node of each tree."""
+    pars = _deep_branched_trees()[name]
+    for p in pars:
+        assert all(-1 <= x < i for i, x in enumerate(p)) and len(p) <= 64
+    assert max(int(W.depths_of(p).max()) for p in pars) > 8
+    paths = []
+    for p in pars:
+        d = W.depths_of(p)
+        n = int(np.flatnonzero(d == d.max())[0])
+        paths.append(O.path_to(p, n))
+    w = W.synthetic(pars, H=4, dk=128, dv=128, seed=len(name) * 7 + len(pars),
+                    paths=paths, log_a_mean=-5.0, name=name)
+    _full_check(w, kernel)

@@ -42,11 +42,22 @@ def test_noalloc_matches_tree_verify_twice(idx, kernel):
         out = torch.full_like(ref_out, float("nan"))
         U = torch.full_like(ref_U, float("nan"))
         scratch = ctypes.c_void_p()
+        torch.cuda.synchronize()
+        free_before, _ = torch.cuda.mem_get_info()
+        torch.cuda.reset_peak_memory_stats()
+        allocated = torch.cuda.memory_allocated()
         st = fn(ctypes.byref(prob), d["q"].data_ptr(), d["k"].data_ptr(), d["v"].data_ptr(),
                 d["log_a"].data_ptr(), d["b"].data_ptr(), d["parent"].data_ptr(),
                 d["node_offsets"].data_ptr(), d["S_root"].data_ptr(), out.data_ptr(),
                 U.data_ptr(), ctypes.byref(scratch), stream)
+        torch.cuda.synchronize()
         assert st == 0, L.binding.status_string(st)
+        if call == 1:
+            # the call itself allocates nothing: neither through torch's allocator nor
+            # anywhere else on the device (the first call may load the module image)
+            assert torch.cuda.max_memory_allocated() == allocated
+            free_after, _ = torch.cuda.mem_get_info()
+            assert free_before - free_after < 2 << 20, (free_before, free_after)
         assert scratch.value, "the static scratch address is reported"
         assert L.lib().tv_get_status(scratch, stream) == 0
         torch.cuda.synchronize()
