@@ -364,8 +364,9 @@ def run_b200(args, workloads):
         vb, cb = verify_bytes(w0), commit_bytes(w0)
         v_avg = statistics.mean(verify_ms) / 1e3
         c_avg = statistics.mean(commit_ms) / 1e3
-        tc = args.kernel != "simt" and w0.max_nodes <= 64
-        kfile, kname = ("verify_tc.cu", "verify_tc") if tc else ("verify_simt.cu", "verify_simt")
+        tc = args.kernel != "simt"
+        kfile, kname = ((("verify_tc.cu", "verify_tc") if w0.max_nodes <= 64 else
+                         ("verify_tcw.cu", "verify_tcw")) if tc else ("verify_simt.cu", "verify_simt"))
         achieved = vb / v_avg / 1e9
         line = {
             "metric": METRIC, "value": value, "unit": "nodes/s", "n_gpus": world,

@@ -108,7 +108,9 @@ typedef enum { TV_KERNEL_AUTO = 0, TV_KERNEL_TC = 1, TV_KERNEL_SIMT = 2 } tv_ker
  *   in_dtype     storage type of q, k, v (TV_F32 or TV_BF16)
  *   out_dtype    storage type of out (TV_F32, or TV_BF16 when in_dtype is TV_BF16)
  *   kernel       tv_kernel (verify only)
- * The tensor-core kernel needs in_dtype = TV_BF16, dk = dv = 128 and max_nodes <= 64. */
+ * The tensor-core kernels need in_dtype = TV_BF16 and dk = dv = 128 (any max_nodes: one
+ * kernel takes trees of up to 64 nodes, another wider ones; trees deeper than 16 nodes
+ * in the wider kernel are verified on CUDA cores inside the same launch). */
 typedef struct {
   int32_t B, H, dk, dv;
   int32_t total_nodes, max_nodes, max_path;

@@ -35,7 +35,7 @@ bool ptr_ok(const void *ptr) { return ptr && aligned16(ptr); }
 
 bool tc_supports(const tv_problem *p) {
   return p->in_dtype == TV_BF16 && p->dk == 128 && p->dv == 128 &&
-         p->max_nodes <= verify_tc_max_nodes();
+         p->max_nodes <= verify_tcw_max_nodes();
 }
 
 thread_local cudaError_t g_last_cuda = cudaSuccess;
@@ -109,7 +109,10 @@ tv_status tv_tree_verify(const tv_problem *p, const void *q, const void *k, cons
   a.B = p->B; a.H = p->H; a.dk = p->dk; a.dv = p->dv; a.T = p->total_nodes;
   a.max_nodes = p->max_nodes;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (use_tc) return from_cuda(launch_verify_tc(a, p->mode, p->out_dtype, s));
+  if (use_tc)   // trees of up to 64 nodes, and wider trees, have one tensor-core kernel each
+    return from_cuda(p->max_nodes <= verify_tc_max_nodes()
+                         ? launch_verify_tc(a, p->mode, p->out_dtype, s)
+                         : launch_verify_tcw(a, p->mode, p->out_dtype, s));
   return from_cuda(launch_verify_simt(a, p->mode, p->in_dtype, p->out_dtype, s));
 }
 

@@ -72,6 +72,8 @@ cudaError_t launch_verify_simt(const VerifyArgs &a, int mode, int in_dtype, int 
                                cudaStream_t st);
 int verify_tc_max_nodes();
 cudaError_t launch_verify_tc(const VerifyArgs &a, int mode, int out_dtype, cudaStream_t st);
+int verify_tcw_max_nodes();
+cudaError_t launch_verify_tcw(const VerifyArgs &a, int mode, int out_dtype, cudaStream_t st);
 int commit_max_path_width();
 cudaError_t launch_commit(const CommitArgs &a, int in_dtype, cudaStream_t st);
 cudaError_t launch_meta(const MetaArgs &a, cudaStream_t st);

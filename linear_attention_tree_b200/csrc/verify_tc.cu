@@ -39,11 +39,8 @@
 //
 // Every wait on an mbarrier is bounded; a wait that runs out records TV_ERR_TIMEOUT on
 // the status word, the CTA drains what it issued, frees its tensor memory and returns.
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
 #include "tc_ptx.cuh"
+#include "tmaps.cuh"
 #include "tv_internal.cuh"
 
 namespace tv {
@@ -593,38 +590,11 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 // ---- host side ------------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// [T][H][128] bf16 viewed as a 3-D tensor (128, H, T); box = 64 elements x 1 head x 64 nodes.
-bool make_map(CUtensorMap *m, const void *ptr, int H, int T) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)T};
-  cuuint64_t strides[2] = {128 * 2, (cuuint64_t)H * 128 * 2};
-  cuuint32_t box[3] = {64, 1, (cuuint32_t)kTile};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <bool kGdn, typename Tout>
 cudaError_t launch_tc_t(const VerifyArgs &a, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, a.q, a.H, a.T) || !make_map(&mk, a.k, a.H, a.T) ||
-      !make_map(&mv, a.v, a.H, a.T))
+  if (!make_node_map(&mq, a.q, a.H, a.T, kTile) || !make_node_map(&mk, a.k, a.H, a.T, kTile) ||
+      !make_node_map(&mv, a.v, a.H, a.T, kTile))
     return cudaErrorInvalidValue;
   auto kern = verify_tc_kernel<kGdn, Tout>;
   cudaError_t e =

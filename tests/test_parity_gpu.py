@@ -224,3 +224,55 @@ def test_deep_branched_trees(name, kernel):
     w = W.synthetic(pars, H=4, dk=128, dv=128, seed=len(name) * 7 + len(pars),
                     paths=paths, log_a_mean=-5.0, name=name)
     _full_check(w, kernel)
+
+
+def _chain_with_depth(n, depth, seed):
+    """n nodes: a root chain of `depth` nodes, the rest attached at random above depth - 1,
+    so the deepest path has exactly `depth` nodes."""
+    rng = np.random.default_rng(seed)
+    par = [i - 1 for i in range(depth)]
+    dep = list(range(1, depth + 1))
+    for i in range(depth, n):
+        while True:
+            p = int(rng.integers(-1, i))
+            d = 1 if p < 0 else dep[p] + 1
+            if d <= depth:
+                break
+        par.append(p)
+        dep.append(d)
+    return par
+
+
+@pytest.mark.parametrize("kernel", ["tc", "simt"])
+@pytest.mark.parametrize("counts", [[256, 65, 1, 0, 130], [200, 77], [129, 128, 64, 63]])
+def test_wide_ragged_full(kernel, counts):
+    """Batches whose largest tree is wider than 64 nodes (the wide tensor-core kernel),
+    ragged down to empty and one-node trees, compared in full."""
+    w = W.synthetic(_ragged(sum(counts) % 97, counts, max_depth=10, fmax=6), H=3, dk=128,
+                    dv=128, seed=len(counts) * 31 + sum(counts), name="wide-ragged",
+                    log_a_mean=-6.0)
+    _full_check(w, kernel)
+
+
+@pytest.mark.parametrize("depth", [15, 16, 17, 40])
+def test_wide_depth_boundary_tc(depth):
+    """Paths of up to 16 nodes stay on the wide kernel's tensor-core path; deeper trees take
+    the CUDA-core algorithm inside the same launch.  Both sides of the boundary, with a
+    shallow wide tree in the same batch."""
+    pars = [_chain_with_depth(150, depth, depth), W.frontier_tree(5 + depth, 90, 8, 4)[0]]
+    paths = [O.path_to(p, int(np.argmax(W.depths_of(p)))) for p in pars]
+    w = W.synthetic(pars, H=2, dk=128, dv=128, seed=depth, paths=paths, log_a_mean=-6.0,
+                    name=f"depth{depth}")
+    assert int(W.depths_of(pars[0]).max()) == depth
+    _full_check(w, "tc")
+
+
+def test_wide_scalar_and_bf16_output():
+    pars = _ragged(11, [180, 90], max_depth=9, fmax=5)
+    w = W.synthetic(pars, H=2, dk=128, dv=128, seed=11, mode="scalar", log_a_mean=-3.0)
+    _full_check(w, "tc")
+    w = W.synthetic(pars, H=2, dk=128, dv=128, seed=12, out_dtype="bf16", log_a_mean=-6.0)
+    res, _ = run(w, kernel="tc")
+    o, _ = O.tree_verify(w)
+    rms = np.sqrt(np.mean(o ** 2))
+    assert np.all(np.abs(res["o"] - o) <= TOL["bf16"] * rms + 2.0 ** -9 * np.abs(o))
