@@ -14,6 +14,10 @@ kernels, so each kernel's CTAs can become resident while the previous kernel dra
 are launched with programmatic stream serialisation).  Per-kernel durations, used for the
 roofline figures, come from a second timed pass with an event before and after every
 kernel; those events keep the kernels apart, so that pass is slower than the step rate.
+Also reported: verify alone launched back to back, the ragged (B=128, 8..48 nodes) and
+wide (B=8, 256 nodes) workloads timed per launch, and the float64 oracle on this host's
+cores, whose values for the whole workload are compared with this run's GPU outputs
+(the run fails if any element is off by more than 2e-2 of the tensor's RMS).
 
 Usage:
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
@@ -187,19 +191,29 @@ def run_reference(args, w):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
-    # about two minutes of oracle work for the whole run, at least one node per step
-    per_node_s = 0.035
-    k = int(min(w.T, max(1, 120.0 / ((args.steps + args.warmup) * per_node_s))))
-    for i in range(args.warmup):
-        oracle_nodes(w, [(i * k + j) % w.T for j in range(k)])
-    total_nodes, total_t = 0, 0.0
-    for i in range(args.steps):
-        n, dt = oracle_nodes(w, [((args.warmup + i) * k + j) % w.T for j in range(k)])
-        total_nodes += n
-        total_t += dt
+    from oracle.pool import oracle_rows, start_pool
+    cores = _cores()
+    pool = start_pool(cores)
+    try:
+        # about two minutes of oracle work for the whole run on the host's cores, at least
+        # one node per step
+        per_node_s = 0.035 / cores
+        k = int(min(w.T, max(1, 120.0 / ((args.steps + args.warmup) * per_node_s))))
+        for i in range(args.warmup):
+            oracle_rows(WORKLOAD_IDX, 0, [(i * k + j) % w.T for j in range(k)], pool)
+        total_nodes, total_t = 0, 0.0
+        for i in range(args.steps):
+            t0 = time.perf_counter()
+            total_nodes += oracle_rows(WORKLOAD_IDX, 0,
+                                       [((args.warmup + i) * k + j) % w.T for j in range(k)], pool)
+            total_t += time.perf_counter() - t0
+    finally:
+        pool.close()
+        pool.join()
     value = total_nodes / total_t
     sample = (f"{args.steps} step(s) of {k} consecutive node(s) x {w.H} heads of the workload "
-              f"(verify of each node, commit of each sequence completed), fp64 numpy, one BLAS thread")
+              f"(verify of each node, commit of each sequence completed), fp64 numpy, "
+              f"{cores} worker processes of one BLAS thread each")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "nodes/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -207,13 +221,56 @@ def run_reference(args, w):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "nodes_per_tree": 64,
                    "dk": w.dk, "dv": w.dv, "seed": 0},
-        "cpu_baseline": {"value": value, "unit": "nodes/s", "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "nodes/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "nodes/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def _cores() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
+
+
+def cpu_baseline_and_self_check(w, got, tol=2e-2):
+    """The float64 oracle timed on this host (one core on a sample, then every core on the
+    whole workload), and the whole workload's oracle values compared with this run's GPU
+    outputs for the same inputs (o, U and S_new, element by element, max|err| <= tol * RMS).
+    ``got`` = (o, U, S_new) as float64 arrays.  Raises if the outputs are off."""
+    from oracle.pool import oracle_config, start_pool
+    n1, dt1 = oracle_nodes(w, list(range(10 * 64)))
+    cores = _cores()
+    pool = start_pool(cores)
+    try:
+        t0 = time.perf_counter()
+        _, o, U, S_new = oracle_config(WORKLOAD_IDX, 0, pool=pool)
+        dt = time.perf_counter() - t0
+    finally:
+        pool.close()
+        pool.join()
+    check = {}
+    for name, g, want in (("o", got[0], o), ("U", got[1], U), ("S_new", got[2], S_new)):
+        rms = float(np.sqrt(np.mean(want ** 2)))
+        err = float(np.max(np.abs(g - want)))
+        check[name] = {"max_err_over_rms": err / rms, "elements": int(want.size)}
+        if not err <= tol * rms:
+            raise RuntimeError(f"self-check failed: {name} max|err| {err:.3e} > {tol} * RMS {rms:.3e}")
+    return {
+        "value": w.T / dt, "unit": "nodes/s", "cores": cores, "kind": "oracle",
+        "sample": (f"the whole workload (seed 0: {w.T} nodes x {w.H} heads, verify, and the "
+                   f"commit of all {w.B} sequences), fp64 numpy, {cores} worker processes of "
+                   "one BLAS thread each"),
+        "seconds": dt,
+        "single_core": {"value": n1 / dt1, "unit": "nodes/s", "cores": 1, "seconds": dt1,
+                        "sample": "sequences 0-9 (10 x 64 nodes x 32 heads), verify + commit"},
+        "self_check": dict(check, tolerance=f"max|err| <= {tol} * RMS(oracle), every element",
+                           outputs="this run's GPU outputs for input set 0"),
+    }
 
 
 # --------------------------------------------------------------------------------- GPU leg
@@ -296,6 +353,44 @@ def run_b200(args, workloads):
     st = L.get_status(ws)
     if st != 0:
         raise RuntimeError(f"device status {st} after the timed region")
+
+    # ---- verify alone, launched back to back (rotating inputs), one event pair around all
+    n_b2b = min(max(args.steps, 20), 2000)
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b0.record(stream)
+    for i in range(n_b2b):
+        d, (o, U, S_new) = sets[i % N_SETS], outs[i % N_SETS]
+        L.tree_verify(d["q"], d["k"], d["v"], d["log_a"], d["b"], d["parent"],
+                      d["node_offsets"], d["S_root"], max_nodes=w0.max_nodes, out=o, U=U,
+                      workspace=ws, kernel=args.kernel)
+    b1.record(stream)
+    torch.cuda.synchronize(dev)
+    b2b_s = b0.elapsed_time(b1) / 1e3 / n_b2b
+
+    # ---- decode steps through the fused entry point: the previous set's commit and this
+    # set's verify in one launch, the state updated in place
+    S_run = sets[0]["S_root"].clone()
+    n_fused = min(max(args.steps, 20), 2000)
+
+    def fused_step(i):
+        dp, dn = sets[(i - 1) % N_SETS], sets[i % N_SETS]
+        L.tree_commit_verify(outs[(i - 1) % N_SETS][1], dp["k"], dp["log_a"], dp["node_offsets"],
+                             dp["accepted_path"], S_run, dn["q"], dn["k"], dn["v"], dn["log_a"],
+                             dn["b"], dn["parent"], dn["node_offsets"],
+                             max_nodes_prev=w0.max_nodes, max_nodes=w0.max_nodes, S_new=S_run,
+                             out=outs[i % N_SETS][0], U=outs[i % N_SETS][1], workspace=ws,
+                             kernel=args.kernel)
+    for i in range(1, 6):
+        fused_step(i)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for i in range(6, 6 + n_fused):
+        fused_step(i)
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    fused_s = f0.elapsed_time(f1) / 1e3 / n_fused
+    if L.get_status(ws) != 0:
+        raise RuntimeError("device status after the fused decode steps")
 
     # ---- end to end through the public API: pinned host inputs in, results out
     host = [to_device(w, "cpu", pin=True) for w in workloads]
@@ -396,18 +491,82 @@ def run_b200(args, workloads):
             "gpu_launches": 2 * args.steps,
             "clocks": clk,
         }
+        line["roofline"]["region"] = ("tv_tree_verify alone: CUDA events around each launch in "
+                                      "the per-kernel pass (the figure the 60% bar applies to); "
+                                      "value is the verify + commit step rate")
+        line["verify_back_to_back"] = {
+            "us_per_launch": 1e6 * b2b_s, "nodes_per_s": T / b2b_s,
+            "frac_of_measured": vb / b2b_s / 1e9 / peak, "frac_of_8TBps": vb / b2b_s / 1e9 / NOMINAL_HBM_GBS,
+            "how": f"{n_b2b} verify launches back to back over the rotating sets, one event pair"}
+        fb = vb + cb - w0.B * w0.H * w0.dk * w0.dv * 4      # S_root read once, not twice
+        line["fused_decode_step"] = {
+            "us_per_step": 1e6 * fused_s, "nodes_per_s": T / fused_s,
+            "algorithmic_bytes_per_step": fb, "achieved_GBps": fb / fused_s / 1e9,
+            "frac_of_measured": fb / fused_s / 1e9 / peak,
+            "how": (f"{n_fused} calls of tv_tree_commit_verify back to back (commit of the "
+                    "previous set's accepted paths + verify of this set, one launch, state in "
+                    "place), one event pair; compare ms_per_step (two launches per step)")}
+        if world == 1 and not args.other_configs_off:
+            line["other_workloads"] = other_workloads(args, L, dev, peak)
         if world == 1 and not args.no_cpu_baseline:
-            n, dt = oracle_nodes(workloads[0], list(range(10 * 64)))
-            line["cpu_baseline"] = {
-                "value": n / dt, "unit": "nodes/s", "cores": 1, "kind": "oracle",
-                "sample": "sequences 0-9 (10 x 64 nodes x 32 heads) of the workload, verify + "
-                          "commit, fp64 numpy, one BLAS thread", "seconds": dt}
+            got = tuple(t.float().cpu().numpy().astype(np.float64) for t in outs[0])
+            line["cpu_baseline"] = cpu_baseline_and_self_check(workloads[0], got)
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def other_workloads(args, L, dev, peak) -> dict:
+    """Per-launch verify timing of the ragged (config 4) and wide-tree (config 5) workloads:
+    rotating input sets, CUDA events around each launch."""
+    import torch
+    from linear_attention_tree_b200 import workloads as W
+    from linear_attention_tree_b200.tensors import to_device
+    res = {}
+    for idx, label in ((4, "gdn ragged trees B=128 H=32, 8..48 nodes, budget 3072, depth<=7"),
+                       (5, "gdn wide trees B=8 H=32, 256 nodes, depth<=10, branching<=8")):
+        ws_ = [W.config(idx, s) for s in range(N_SETS)]
+        ds = [to_device(x, dev) for x in ws_]
+        w = ws_[0]
+        odt = torch.float32 if w.out_dtype == "f32" else torch.bfloat16
+        outs = [(torch.empty((x.T, x.H, x.dv), dtype=odt, device=dev),
+                 torch.empty((x.T, x.H, x.dv), dtype=torch.float32, device=dev)) for x in ws_]
+        ws = L.new_workspace(L.make_problem(w.B, w.H, w.dk, w.dv, w.T, w.max_nodes, w.max_path), dev)
+
+        def one(i):
+            d, (o, U), x = ds[i % N_SETS], outs[i % N_SETS], ws_[i % N_SETS]
+            L.tree_verify(d["q"], d["k"], d["v"], d["log_a"], d["b"], d["parent"],
+                          d["node_offsets"], d["S_root"], max_nodes=x.max_nodes, out=o, U=U,
+                          workspace=ws, kernel=args.kernel)
+        for i in range(10):
+            one(i)
+        n = 60
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n)]
+        for i, (e0, e1) in enumerate(ev):
+            e0.record()
+            one(i)
+            e1.record()
+        torch.cuda.synchronize(dev)
+        if L.get_status(ws) != 0:
+            raise RuntimeError(f"device status after workload {idx}")
+        t = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev) / 1e3
+        vb = statistics.mean(verify_bytes(x) for x in ws_)
+        T = statistics.mean(x.T for x in ws_)
+        kname = ("verify_tc" if w.max_nodes <= 64 else "verify_tcw") if args.kernel != "simt" \
+            else "verify_simt"
+        res[f"config{idx}"] = {
+            "workload": label, "kernel": kname, "verify_us": 1e6 * t,
+            "verify_nodes_per_s": T / t, "algorithmic_bytes_per_launch": int(vb),
+            "achieved_GBps": vb / t / 1e9, "frac_of_measured": vb / t / 1e9 / peak,
+            "frac_of_8TBps": vb / t / 1e9 / NOMINAL_HBM_GBS,
+            "timing": f"CUDA events around each of {n} launches, {N_SETS} rotating input sets"}
+        del ds, outs
+        torch.cuda.empty_cache()
+    return res
 
 
 def main(argv=None):
@@ -418,6 +577,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--kernel", choices=["auto", "tc", "simt"], default="auto")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--other-configs-off", action="store_true",
+                    help="skip the per-launch timing of the ragged and wide-tree workloads")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

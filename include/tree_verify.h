@@ -160,6 +160,37 @@ TV_API tv_status tv_tree_commit(const tv_problem *p, const float *U, const void 
                          const int32_t *parent, float *S_new, void *workspace,
                          size_t workspace_bytes, tv_stream_t stream);
 
+/* One decode step's commit followed by the next step's verify, against the committed state:
+ *   S_new = tv_tree_commit(prev, U_prev, k_prev, log_a_prev, S_root, node_offsets_prev,
+ *                          accepted_path, parent_prev)
+ *   (out, U) = tv_tree_verify(next, q, k, v, log_a, b, parent, node_offsets, S_root = S_new)
+ * with the results of those two calls, in one pass over the state where the shapes allow it
+ * (the committed state is rebuilt in registers and verified against without being read back
+ * from memory; Twig abstract: only the accepted state is rebuilt; Bole summary, worked
+ * example "具体技术细节示例": only S_c3 is rebuilt, and decoding goes on from it).  That
+ * single pass is taken for bf16 inputs with dk = dv = 128, next->max_nodes <= 64,
+ * prev->max_path <= 32 and next->kernel AUTO or TC; otherwise the two kernels run in turn.
+ *   prev       the previous step's problem (its max_path = row width of accepted_path); B, H,
+ *              dk and dv must equal next's
+ *   U_prev, k_prev, log_a_prev, node_offsets_prev, parent_prev (may be NULL), accepted_path:
+ *              as in tv_tree_commit, for the previous step's tree          (device, read)
+ *   S_root     [B][H][dv][dk] fp32, the state before the commit            (device, read)
+ *   S_new      [B][H][dv][dk] fp32; may be S_root itself, must not partially overlap it
+ *                                                                           (device, written)
+ *   next, q, k, v, log_a, b, parent, node_offsets: as in tv_tree_verify, for the next tree
+ *   out, U     as in tv_tree_verify; U must not overlap U_prev              (device, written)
+ * A sequence whose next tree is empty or malformed is still committed. */
+TV_API tv_status tv_tree_commit_verify(const tv_problem *prev, const float *U_prev,
+                                       const void *k_prev, const float *log_a_prev,
+                                       const int32_t *node_offsets_prev,
+                                       const int32_t *accepted_path, const int32_t *parent_prev,
+                                       const float *S_root, float *S_new, const tv_problem *next,
+                                       const void *q, const void *k, const void *v,
+                                       const float *log_a, const float *b, const int32_t *parent,
+                                       const int32_t *node_offsets, void *out, float *U,
+                                       void *workspace, size_t workspace_bytes,
+                                       tv_stream_t stream);
+
 /* Tree metadata of every node (exported for tests and for callers that cache it):
  *   depth  [T] int32: tokens on the root->n path (first-level node = 1)
  *   anc    [T][W] uint64, W = ceil(max_nodes/64): bit (i%64) of word i/64 is set iff local

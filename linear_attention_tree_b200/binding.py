@@ -9,6 +9,7 @@ Python name  -> C entry point
   tree_verify     tv_tree_verify
   tree_commit     tv_tree_commit
   tree_meta       tv_tree_meta
+  tree_commit_verify tv_tree_commit_verify
   workspace_size  tv_workspace_size
   get_status      tv_get_status
   selftest_timeout tv_selftest_timeout
@@ -30,6 +31,7 @@ MODE = {"gdn": 0, "scalar": 1}
 DTYPE = {torch.float32: 0, torch.bfloat16: 1}
 KERNEL = {"auto": 0, "tc": 1, "simt": 2}
 EXPORTS = ("tv_workspace_size", "tv_tree_verify", "tv_tree_commit", "tv_tree_meta",
+           "tv_tree_commit_verify",
            "tv_get_status", "tv_status_string", "tv_last_cuda_error", "tv_version",
            "tv_selftest_timeout")
 
@@ -69,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.tv_tree_commit.argtypes = [P] + [vp] * 9 + [ctypes.c_size_t, vp]
         L.tv_tree_commit.restype = ctypes.c_int
         L.tv_tree_meta.argtypes = [P] + [vp] * 7 + [ctypes.c_size_t, vp]
+        L.tv_tree_commit_verify.argtypes = [P] + [vp] * 8 + [P] + [vp] * 10 + [ctypes.c_size_t, vp]
+        L.tv_tree_commit_verify.restype = ctypes.c_int
         L.tv_tree_meta.restype = ctypes.c_int
         L.tv_get_status.argtypes = [vp, vp]
         L.tv_get_status.restype = ctypes.c_int
@@ -208,6 +212,62 @@ def tree_commit(U, k, log_a, S_root, node_offsets, accepted_path, *, max_nodes: 
                               _stream(stream))
     _check(st, "tv_tree_commit")
     return S_new
+
+
+def tree_commit_verify(U_prev, k_prev, log_a_prev, node_offsets_prev, accepted_path, S_root,
+                       q, k, v, log_a, b, parent, node_offsets, *, max_nodes_prev: int,
+                       max_nodes: int, parent_prev=None, S_new=None, out=None, U=None,
+                       mode: str = "gdn", out_dtype=None, workspace=None, kernel: str = "auto",
+                       stream=None):
+    """The previous step's commit and the next tree's verify against the committed state;
+    returns (S_new, out, U).  ``S_new`` may be ``S_root`` (in place); ``U`` must not be
+    ``U_prev``.  Argument meanings as in `tree_commit` (previous tree) and `tree_verify`
+    (next tree)."""
+    Tp, H, dv = U_prev.shape
+    dk = k_prev.shape[2]
+    B = node_offsets.shape[0] - 1
+    T = q.shape[0]
+    dev = q.device
+    out_dtype = out_dtype or q.dtype
+    if S_new is None:
+        S_new = torch.empty_like(S_root)
+    if out is None:
+        out = torch.empty((T, H, dv), dtype=out_dtype, device=dev)
+    if U is None:
+        U = torch.empty((T, H, dv), dtype=torch.float32, device=dev)
+    max_path = accepted_path.shape[1]
+    prev = make_problem(B, H, dk, dv, Tp, max_nodes_prev, max_path, mode, k_prev.dtype,
+                        k_prev.dtype)
+    nxt = make_problem(B, H, dk, dv, T, max_nodes, 1, mode, q.dtype, out.dtype, kernel)
+    if workspace is None:
+        workspace = new_workspace(nxt, dev)
+    fdt = torch.float32
+    args = [
+        _ptr(U_prev, "U_prev", fdt, (Tp, H, dv), dev),
+        _ptr(k_prev, "k_prev", (torch.float32, torch.bfloat16), (Tp, H, dk), dev),
+        _ptr(log_a_prev, "log_a_prev", fdt, (Tp, H), dev),
+        _ptr(node_offsets_prev, "node_offsets_prev", torch.int32, (B + 1,), dev),
+        _ptr(accepted_path, "accepted_path", torch.int32, (B, max_path), dev),
+        _ptr(parent_prev, "parent_prev", torch.int32, (Tp,), dev),
+        _ptr(S_root, "S_root", fdt, (B, H, dv, dk), dev),
+        _ptr(S_new, "S_new", fdt, (B, H, dv, dk), dev),
+    ]
+    args2 = [
+        _ptr(q, "q", (torch.float32, torch.bfloat16), (T, H, dk), dev),
+        _ptr(k, "k", q.dtype, (T, H, dk), dev),
+        _ptr(v, "v", q.dtype, (T, H, dv), dev),
+        _ptr(log_a, "log_a", fdt, (T, H), dev),
+        _ptr(b, "b", fdt, (T, H), dev),
+        _ptr(parent, "parent", torch.int32, (T,), dev),
+        _ptr(node_offsets, "node_offsets", torch.int32, (B + 1,), dev),
+        _ptr(out, "out", (torch.float32, torch.bfloat16), (T, H, dv), dev),
+        _ptr(U, "U", fdt, (T, H, dv), dev),
+        _ptr(workspace, "workspace", torch.uint8, None, dev),
+    ]
+    st = lib().tv_tree_commit_verify(ctypes.byref(prev), *args, ctypes.byref(nxt), *args2,
+                                     ctypes.c_size_t(workspace.numel()), _stream(stream))
+    _check(st, "tv_tree_commit_verify")
+    return S_new, out, U
 
 
 def tree_meta(parent, node_offsets, log_a, *, max_nodes: int, workspace=None, stream=None):

@@ -144,6 +144,73 @@ tv_status tv_tree_commit(const tv_problem *p, const float *U, const void *k,
   return from_cuda(launch_commit(a, p->in_dtype, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+tv_status tv_tree_commit_verify(const tv_problem *prev, const float *U_prev, const void *k_prev,
+                                const float *log_a_prev, const int32_t *node_offsets_prev,
+                                const int32_t *accepted_path, const int32_t *parent_prev,
+                                const float *S_root, float *S_new, const tv_problem *next,
+                                const void *q, const void *k, const void *v, const float *log_a,
+                                const float *b, const int32_t *parent,
+                                const int32_t *node_offsets, void *out, float *U, void *workspace,
+                                size_t workspace_bytes, tv_stream_t stream) {
+  tv_status st = check_problem(prev);
+  if (st == TV_OK) st = check_problem(next);
+  if (st != TV_OK) return st;
+  if (prev->B != next->B || prev->H != next->H || prev->dk != next->dk || prev->dv != next->dv)
+    return TV_ERR_INVALID_ARG;
+  if (prev->max_path < 1) return TV_ERR_INVALID_ARG;
+  if (prev->max_path > commit_max_path_width()) return TV_ERR_UNSUPPORTED;
+  if (!ptr_ok(U_prev) || !ptr_ok(k_prev) || !ptr_ok(log_a_prev) || !ptr_ok(node_offsets_prev) ||
+      !ptr_ok(accepted_path) || !ptr_ok(S_root) || !ptr_ok(S_new) || !ptr_ok(q) || !ptr_ok(k) ||
+      !ptr_ok(v) || !ptr_ok(log_a) || !ptr_ok(parent) || !ptr_ok(node_offsets) || !ptr_ok(out) ||
+      !ptr_ok(U) || !ptr_ok(workspace))
+    return TV_ERR_INVALID_ARG;
+  if (parent_prev && !aligned16(parent_prev)) return TV_ERR_INVALID_ARG;
+  if (next->mode == TV_MODE_GDN ? !ptr_ok(b) : (b && !aligned16(b))) return TV_ERR_INVALID_ARG;
+  if (workspace_bytes < kWorkspaceBytes) return TV_ERR_INVALID_ARG;
+  const size_t state_bytes = (size_t)next->B * next->H * next->dv * next->dk * sizeof(float);
+  const char *a0 = reinterpret_cast<const char *>(S_root), *b0 = reinterpret_cast<const char *>(S_new);
+  if (a0 != b0 && a0 < b0 + state_bytes && b0 < a0 + state_bytes) return TV_ERR_INVALID_ARG;
+  // the new pseudo-values must not overwrite the previous ones while they are read
+  const size_t u_prev_bytes = (size_t)prev->total_nodes * prev->H * prev->dv * sizeof(float);
+  const size_t u_bytes = (size_t)next->total_nodes * next->H * next->dv * sizeof(float);
+  const char *c0 = reinterpret_cast<const char *>(U_prev), *d0 = reinterpret_cast<const char *>(U);
+  if (u_prev_bytes && u_bytes && c0 < d0 + u_bytes && d0 < c0 + u_prev_bytes) return TV_ERR_INVALID_ARG;
+  if (next->kernel == TV_KERNEL_TC && !tc_supports(next)) return TV_ERR_UNSUPPORTED;
+  if (next->B == 0) return TV_OK;
+  VerifyArgs a;
+  a.q = q; a.k = k; a.v = v; a.log_a = log_a; a.b = b; a.parent = parent;
+  a.node_offsets = node_offsets; a.S_root = S_root; a.out = out; a.U = U;
+  a.ws = static_cast<int *>(workspace);
+  a.B = next->B; a.H = next->H; a.dk = next->dk; a.dv = next->dv; a.T = next->total_nodes;
+  a.max_nodes = next->max_nodes;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool fused = next->kernel != TV_KERNEL_SIMT && tc_supports(next) &&
+                     next->max_nodes <= verify_tc_max_nodes() && prev->in_dtype == TV_BF16 &&
+                     prev->max_path <= fused_max_path();
+  if (fused) {
+    FuseArgs f;
+    f.U = U_prev; f.k = k_prev; f.log_a = log_a_prev; f.node_offsets = node_offsets_prev;
+    f.accepted_path = accepted_path; f.parent = parent_prev; f.S_new = S_new;
+    f.T = prev->total_nodes; f.max_nodes = prev->max_nodes; f.max_path = prev->max_path;
+    return from_cuda(launch_commit_verify_tc(a, f, next->mode, next->out_dtype, s));
+  }
+  // otherwise the commit, then the verify on its result: two launches, same results
+  CommitArgs c;
+  c.U = U_prev; c.k = k_prev; c.log_a = log_a_prev; c.S_root = S_root;
+  c.node_offsets = node_offsets_prev; c.accepted_path = accepted_path; c.parent = parent_prev;
+  c.S_new = S_new; c.ws = a.ws;
+  c.B = prev->B; c.H = prev->H; c.dk = prev->dk; c.dv = prev->dv; c.T = prev->total_nodes;
+  c.max_nodes = prev->max_nodes; c.max_path = prev->max_path;
+  st = from_cuda(launch_commit(c, prev->in_dtype, s));
+  if (st != TV_OK) return st;
+  a.S_root = S_new;
+  if (next->kernel != TV_KERNEL_SIMT && tc_supports(next))
+    return from_cuda(next->max_nodes <= verify_tc_max_nodes()
+                         ? launch_verify_tc(a, next->mode, next->out_dtype, s)
+                         : launch_verify_tcw(a, next->mode, next->out_dtype, s));
+  return from_cuda(launch_verify_simt(a, next->mode, next->in_dtype, next->out_dtype, s));
+}
+
 tv_status tv_tree_meta(const tv_problem *p, const int32_t *parent,
                        const int32_t *node_offsets, const float *log_a, int32_t *depth,
                        uint64_t *anc, float *cumlog, void *workspace,

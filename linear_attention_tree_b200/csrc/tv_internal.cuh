@@ -52,6 +52,17 @@ struct CommitArgs {
   int B, H, dk, dv, T, max_nodes, max_path;
 };
 
+// The commit that a fused commit + verify launch applies to S_root before verifying: the
+// previous step's tree, its pseudo-values and its accepted paths (one row per sequence).
+struct FuseArgs {
+  const float *U;                    // previous step's U
+  const void *k;                     // previous step's k (bf16)
+  const float *log_a;
+  const int32_t *node_offsets, *accepted_path, *parent;   // parent may be NULL
+  float *S_new;                      // may be S_root
+  int T, max_nodes, max_path;
+};
+
 struct MetaArgs {
   const int32_t *parent, *node_offsets;
   const float *log_a;
@@ -72,6 +83,9 @@ cudaError_t launch_verify_simt(const VerifyArgs &a, int mode, int in_dtype, int 
                                cudaStream_t st);
 int verify_tc_max_nodes();
 cudaError_t launch_verify_tc(const VerifyArgs &a, int mode, int out_dtype, cudaStream_t st);
+int fused_max_path();
+cudaError_t launch_commit_verify_tc(const VerifyArgs &a, const FuseArgs &f, int mode, int out_dtype,
+                                    cudaStream_t st);
 int verify_tcw_max_nodes();
 cudaError_t launch_verify_tcw(const VerifyArgs &a, int mode, int out_dtype, cudaStream_t st);
 int commit_max_path_width();

@@ -53,6 +53,7 @@ constexpr uint32_t kTmemCols = 256;        // two CTAs per SM
 constexpr uint32_t kColGram = 128;         // [Q ; K] . K^T  (lanes = q / k rows)
 constexpr uint32_t kColR = 192;            // R^T            (lanes = value index)
 constexpr uint32_t kSpinLimit = 1u << 22;  // polls before a wait is declared timed out
+constexpr int kFuseMax = 32;               // longest accepted path of a fused commit
 
 // Dynamic shared memory, offsets from a 1024-byte aligned base.
 //   [0, 32K)    [Q ; K]: 128 rows x 128 bf16 as two 64-wide K halves of 16 KiB (TMA swizzled)
@@ -95,6 +96,12 @@ struct Misc {
   __align__(16) float gam[kTile];  // gamma_n
   __align__(16) float bg[kTile];   // b_n gamma_n
   __align__(16) float bq[kTile];   // b_n (copy read as float4)
+  // fused commit of the previous step (kFused): its accepted path for this sequence
+  int f_m, f_lo, f_stat;
+  float f_gam;                     // exp(c_m)
+  int f_prow[kFuseMax];            // root-first path nodes (local to the previous tree)
+  float f_la[kFuseMax];            // log_a of the path nodes, then the prefix sums c_j
+  float f_e[kFuseMax];             // exp(c_m - c_j)
 };
 constexpr int kSmemBytes = kOffMisc + (int)sizeof(Misc) + 1024;
 
@@ -194,6 +201,110 @@ __device__ __noinline__ void row_coefficients_deep(unsigned char *sm, const uint
   }
 }
 
+// ---- fused commit of the previous step ---------------------------------------------------
+// S_new = exp(c_m) S_root + sum_j exp(c_m - c_j) u_{p_j} k_{p_j}^T along the accepted path
+// p_1..p_m of the previous tree (the Bole summary's worked example rebuilds S_c3 this way;
+// with the tree solve's pseudo-values the same form holds for the gated delta rule), applied
+// to the S_root values this CTA holds in registers before it verifies the next tree against
+// S_new.  The u and k rows of the path sit in the bf16 S_root operand region until the
+// operand is written.
+
+// One warp: the previous tree's node range and the accepted-path row of sequence s, checked.
+__device__ __forceinline__ void fuse_gather_path(Misc &ms, const FuseArgs &f, int s, int B,
+                                                 int lane) {
+  const int lo = f.node_offsets[s], hi = f.node_offsets[s + 1];
+  const bool tree_ok = !(lo < 0 || hi < lo || hi > f.T || hi - lo > f.max_nodes ||
+                         (s == 0 && lo != 0) || (s == B - 1 && hi != f.T));
+  const int32_t *row = f.accepted_path + (size_t)s * f.max_path;
+  const int p = lane < f.max_path ? row[lane] : -1;
+  // m = number of leading non-negative entries; after them only -1 may follow
+  const unsigned neg = __ballot_sync(0xffffffffu, lane < f.max_path && p < 0);
+  const int m = neg ? __ffs(neg) - 1 : f.max_path;
+  bool bad = lane < f.max_path && (lane < m ? p >= hi - lo : p != -1);
+  if (lane < m && !bad) ms.f_prow[lane] = p;
+  bad = __any_sync(0xffffffffu, bad) || !tree_ok;
+  if (lane == 0) {
+    ms.f_m = bad ? 0 : m;
+    ms.f_lo = lo;
+    ms.f_stat = bad ? (tree_ok ? TV_ERR_BAD_PATH : TV_ERR_BAD_TREE) : 0;
+  }
+}
+
+// All threads: the u and k rows, log_a and the parent chain of the path entries.
+__device__ __forceinline__ void fuse_load_rows(unsigned char *sm, Misc &ms, const FuseArgs &f,
+                                               int h, int H, int tid) {
+  const int m = ms.f_m, lo = ms.f_lo;
+  float *cu = reinterpret_cast<float *>(sm + kOffS);
+  float *kk = cu + kFuseMax * 128;
+  const __nv_bfloat16 *k = static_cast<const __nv_bfloat16 *>(f.k);
+  for (int idx = tid; idx < m * 128; idx += kThreads) {
+    const size_t node = (size_t)(lo + ms.f_prow[idx >> 7]) * H + h;
+    cu[idx] = f.U[node * 128 + (idx & 127)];
+    kk[idx] = __bfloat162float(k[node * 128 + (idx & 127)]);
+  }
+  if (tid < m) {
+    const int p = ms.f_prow[tid];
+    ms.f_la[tid] = f.log_a[(size_t)(lo + p) * H + h];
+    if (f.parent && f.parent[lo + p] != (tid == 0 ? -1 : ms.f_prow[tid - 1]))
+      ms.f_stat = TV_ERR_BAD_PATH;
+  }
+}
+
+// One thread: fp32 prefix sums c_j root first (the order the verify kernels use for cl), the
+// decay weights, and the status.
+__device__ __forceinline__ void fuse_prefix(Misc &ms, int *ws, int s) {
+  if (ms.f_stat) {
+    set_status(ws, ms.f_stat, s);
+    ms.f_m = 0;
+  }
+  const int m = ms.f_m;
+  float c = 0.f;
+  for (int j = 0; j < m; ++j) {
+    c += ms.f_la[j];
+    ms.f_la[j] = c;
+  }
+  for (int j = 0; j < m; ++j) ms.f_e[j] = expf(c - ms.f_la[j]);
+  ms.f_gam = m ? expf(c) : 1.f;
+}
+
+// All threads: the update on this thread's rows v = tid/16 + 16 j, columns 8 (tid % 16) ..,
+// then S_new streamed out (a malformed path leaves S_root as it is).
+__device__ __forceinline__ void fuse_apply(float4 (&sr)[16], const unsigned char *sm,
+                                           const Misc &ms, float *S_new, int tid) {
+  const int m = ms.f_m, kc = tid & 15;
+  const float g = ms.f_gam;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    sr[i].x *= g; sr[i].y *= g; sr[i].z *= g; sr[i].w *= g;
+  }
+  const float *cu = reinterpret_cast<const float *>(sm + kOffS);
+  const float *kk = cu + kFuseMax * 128;
+  for (int e = 0; e < m; ++e) {
+    const float ee = ms.f_e[e];
+    const float4 ka = *reinterpret_cast<const float4 *>(kk + e * 128 + kc * 8);
+    const float4 kb = *reinterpret_cast<const float4 *>(kk + e * 128 + kc * 8 + 4);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float c = ee * cu[e * 128 + (tid >> 4) + 16 * j];
+      sr[2 * j].x = fmaf(c, ka.x, sr[2 * j].x);
+      sr[2 * j].y = fmaf(c, ka.y, sr[2 * j].y);
+      sr[2 * j].z = fmaf(c, ka.z, sr[2 * j].z);
+      sr[2 * j].w = fmaf(c, ka.w, sr[2 * j].w);
+      sr[2 * j + 1].x = fmaf(c, kb.x, sr[2 * j + 1].x);
+      sr[2 * j + 1].y = fmaf(c, kb.y, sr[2 * j + 1].y);
+      sr[2 * j + 1].z = fmaf(c, kb.z, sr[2 * j + 1].z);
+      sr[2 * j + 1].w = fmaf(c, kb.w, sr[2 * j + 1].w);
+    }
+  }
+  float4 *dst = reinterpret_cast<float4 *>(S_new);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int v = (tid >> 4) + 16 * j;
+    __stcs(dst + v * 32 + kc * 2, sr[2 * j]);
+    __stcs(dst + v * 32 + kc * 2 + 1, sr[2 * j + 1]);
+  }
+}
+
 __device__ __forceinline__ void release_tmem(int warp, uint32_t tmem) {
   ptx::tc_fence_before();
   __syncthreads();
@@ -215,11 +326,11 @@ __device__ __forceinline__ bool wait_all(Misc &ms, uint32_t bar, int tid, int *w
   return ms.flag == 0;
 }
 
-template <bool kGdn, typename Tout>
+template <bool kGdn, typename Tout, bool kFused>
 __global__ void __launch_bounds__(kThreads, 2)
     verify_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, VerifyArgs a,
+                     const __grid_constant__ CUtensorMap tm_v, VerifyArgs a, FuseArgs f,
                      int prefetch_stride) {
   extern __shared__ unsigned char smem_dyn[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
@@ -249,14 +360,25 @@ __global__ void __launch_bounds__(kThreads, 2)
       sr[2 * j + 1] = ldg_first(Sg + v * 32 + kc * 2 + 1);
     }
   }
+  float *const S_new_item = kFused ? f.S_new + ((size_t)s * H + h) * 128 * 128 : nullptr;
   const int lo = a.node_offsets[s], hi = a.node_offsets[s + 1];
-  if (lo < 0 || hi < lo || hi > a.T || hi - lo > a.max_nodes || hi - lo > kTile ||
-      (s == 0 && lo != 0) || (s == a.B - 1 && hi != a.T)) {
-    if (tid == 0) set_status(a.ws, TV_ERR_BAD_TREE, s);
+  const bool range_ok = !(lo < 0 || hi < lo || hi > a.T || hi - lo > a.max_nodes ||
+                          hi - lo > kTile || (s == 0 && lo != 0) || (s == a.B - 1 && hi != a.T));
+  if (!range_ok && tid == 0) set_status(a.ws, TV_ERR_BAD_TREE, s);
+  if (!range_ok || hi == lo) {
+    if (kFused) {
+      // nothing to verify in this sequence: the commit alone
+      if (warp == kThreads / 32 - 1) fuse_gather_path(ms, f, s, a.B, lane);
+      __syncthreads();
+      fuse_load_rows(sm, ms, f, h, H, tid);
+      __syncthreads();
+      if (tid == 0) fuse_prefix(ms, a.ws, s);
+      __syncthreads();
+      fuse_apply(sr, sm, ms, S_new_item, tid);
+    }
     return;
   }
   const int n_nodes = hi - lo;
-  if (n_nodes == 0) return;
 
   const uint32_t sbase = ptx::smem_addr(sm);
   const uint32_t bar_tma = ptx::smem_addr(&ms.bar_tma);
@@ -300,10 +422,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     ms.la[tid] = la;
     ms.bb[tid] = bb;
   }
+  if (kFused && warp == kThreads / 32 - 1) fuse_gather_path(ms, f, s, a.B, lane);
   ptx::tc_fence_before();
   const bool bad_tree = __syncthreads_or(bad) != 0;
   ptx::tc_fence_after();
   const uint32_t tmem = ms.tmem_base;
+  if (kFused) fuse_load_rows(sm, ms, f, h, H, tid);   // landed by the update before step 3's conversion
 
   // ---- 2. Gram MMA once q / k have landed; tree walk ------------------------------------
   if (tid == kThreads - 1) {
@@ -343,10 +467,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     atomicMax(&ms.maxdep, d);
   }
   __syncthreads();
+  if (kFused && tid == 0) fuse_prefix(ms, a.ws, s);
   if (bad_tree || ms.flag != 0) {
     if (tid == 0) {
       set_status(a.ws, bad_tree ? TV_ERR_BAD_TREE : ms.flag, s);
       if (ms.flag == TV_ERR_TIMEOUT) ptx::mbar_wait_bounded(bar_tma, 0, kSpinLimit);
+    }
+    if (kFused) {
+      __syncthreads();
+      fuse_apply(sr, sm, ms, S_new_item, tid);   // the commit does not depend on the next tree
     }
     release_tmem(warp, tmem);
     return;
@@ -386,6 +515,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int j = 0; j < 16; ++j)
         if ((bits >> j) & 1u) pos_major[pos++][gn] = scale * g[j];
     }
+  }
+  if (kFused) {
+    // the previous step's commit, on the values in registers; S_new goes out, and the
+    // verify goes on with it
+    fuse_apply(sr, sm, ms, S_new_item, tid);
+    __syncthreads();   // the path rows are read before the operand overwrites them
   }
   // S_root -> bf16 operand rows (all threads; the loads have long arrived by now)
 #pragma unroll
@@ -590,13 +725,16 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 // ---- host side ------------------------------------------------------------------------
-template <bool kGdn, typename Tout>
-cudaError_t launch_tc_t(const VerifyArgs &a, cudaStream_t st) {
+template <bool kGdn, typename Tout, bool kFused>
+cudaError_t launch_tc_t(const VerifyArgs &a, const FuseArgs &f, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
-  if (!make_node_map(&mq, a.q, a.H, a.T, kTile) || !make_node_map(&mk, a.k, a.H, a.T, kTile) ||
-      !make_node_map(&mv, a.v, a.H, a.T, kTile))
+  // (a next tree with no nodes at all still gets maps over a one-row view: the kernel only
+  // commits then)
+  const int rows = a.T > 0 ? a.T : 1;
+  if (!make_node_map(&mq, a.q, a.H, rows, kTile) || !make_node_map(&mk, a.k, a.H, rows, kTile) ||
+      !make_node_map(&mv, a.v, a.H, rows, kTile))
     return cudaErrorInvalidValue;
-  auto kern = verify_tc_kernel<kGdn, Tout>;
+  auto kern = verify_tc_kernel<kGdn, Tout, kFused>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
@@ -614,19 +752,31 @@ cudaError_t launch_tc_t(const VerifyArgs &a, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, a, 2 * sms);
+  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, a, f, 2 * sms);
 }
 
 }  // namespace
 
 int verify_tc_max_nodes() { return kTile; }
+int fused_max_path() { return kFuseMax; }
 
 cudaError_t launch_verify_tc(const VerifyArgs &a, int mode, int out_dtype, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;   // every tree is empty
   const bool gdn = mode == TV_MODE_GDN;
+  const FuseArgs f = {};
   if (out_dtype == TV_BF16)
-    return gdn ? launch_tc_t<true, __nv_bfloat16>(a, st) : launch_tc_t<false, __nv_bfloat16>(a, st);
-  return gdn ? launch_tc_t<true, float>(a, st) : launch_tc_t<false, float>(a, st);
+    return gdn ? launch_tc_t<true, __nv_bfloat16, false>(a, f, st)
+               : launch_tc_t<false, __nv_bfloat16, false>(a, f, st);
+  return gdn ? launch_tc_t<true, float, false>(a, f, st) : launch_tc_t<false, float, false>(a, f, st);
+}
+
+cudaError_t launch_commit_verify_tc(const VerifyArgs &a, const FuseArgs &f, int mode,
+                                    int out_dtype, cudaStream_t st) {
+  const bool gdn = mode == TV_MODE_GDN;
+  if (out_dtype == TV_BF16)
+    return gdn ? launch_tc_t<true, __nv_bfloat16, true>(a, f, st)
+               : launch_tc_t<false, __nv_bfloat16, true>(a, f, st);
+  return gdn ? launch_tc_t<true, float, true>(a, f, st) : launch_tc_t<false, float, true>(a, f, st);
 }
 
 }  // namespace tv

@@ -125,3 +125,23 @@ def test_selftest_rejects_bad_workspace_before_launching():
     assert f(None, 256, None) == binding.TV_ERR_INVALID_ARG
     assert f(ctypes.c_void_p(0x10004), 256, None) == binding.TV_ERR_INVALID_ARG
     assert f(ctypes.c_void_p(0x10000), 8, None) == binding.TV_ERR_INVALID_ARG
+
+
+def test_commit_verify_checks_its_arguments():
+    """Shapes that differ between the two steps, and new pseudo-values over the previous
+    ones, are refused before anything is enqueued."""
+    import torch
+    fn = L.lib().tv_tree_commit_verify
+    ptr = lambda i: ctypes.c_void_p(0x100000 * (i + 1))
+    prev = L.make_problem(2, 2, 128, 128, 8, 4, 3)
+    nxt = L.make_problem(2, 2, 128, 128, 8, 4, 1)
+    # prev, U_prev, 7 more previous-step pointers, next, q..node_offsets (7), out, U, workspace
+    args = lambda U_prev, U: [ctypes.byref(prev), U_prev] + [ptr(i) for i in range(1, 8)] + \
+        [ctypes.byref(nxt)] + [ptr(i) for i in range(8, 15)] + [ptr(15), U, ptr(18),
+                                                               ctypes.c_size_t(256), None]
+    # U (8 nodes x 2 heads x 128 fp32 = 8 KiB) starting inside U_prev
+    assert fn(*args(ptr(0), ctypes.c_void_p(0x100000 + 4096))) == binding.TV_ERR_INVALID_ARG
+    other = L.make_problem(3, 2, 128, 128, 8, 4, 1)
+    assert fn(ctypes.byref(prev), ptr(0), *[ptr(i) for i in range(1, 8)], ctypes.byref(other),
+              *[ptr(i) for i in range(8, 15)], ptr(15), ptr(17), ptr(18), ctypes.c_size_t(256),
+              None) == binding.TV_ERR_INVALID_ARG

@@ -3,7 +3,7 @@
 Bars: max|err| <= 1e-4 * RMS(oracle tensor) for fp32 inputs, <= 2e-2 * RMS for bf16
 inputs, separately for o, U and S_new.  Every one of the five named workloads is compared
 in full, every node, head and state: 1 and 2 directly, 3-5 against the oracle spread over
-the host's cores (``tests/_oracle_pool.py``), with both kernels and in the launch
+the host's cores (``oracle/pool.py``), with both kernels and in the launch
 configuration the benchmark times.  Smaller trees of every shape class (ragged, empty,
 deep branched, combs, chains) are compared in full as well.
 """
@@ -13,7 +13,7 @@ import pytest
 from linear_attention_tree_b200 import workloads as W
 from oracle import oracle as O
 from tests._gpu_util import TOL, assert_close, run
-from tests._oracle_pool import oracle_config
+from oracle.pool import oracle_config
 
 _FULL = {}
 
