@@ -225,6 +225,28 @@ TV_API tv_status tv_tree_verify_noalloc(const tv_problem *p, const void *q, cons
                                         const float *S_root, void *out, float *U,
                                         void **scratch_out, tv_stream_t stream);
 
+/* The baseline the pages compare against (Twig / Bole abstracts: draft trees verified
+ * sequentially, with the full recurrent state snapshotted for every node), for measuring
+ * speed and transient memory against tv_tree_verify on the same GPU.  Same inputs and
+ * outputs as tv_tree_verify (o and the pseudo-values U, whose meaning is identical), plus
+ *   snapshots  [T][H][dv][dk] fp32: the state of every node, written  (device, written)
+ * Nodes are visited in index order, each starting from its parent's snapshot.  One CTA of
+ * 128 threads per (sequence, head), fp32 arithmetic on CUDA cores. */
+TV_API tv_status tv_snapshot_verify(const tv_problem *p, const void *q, const void *k,
+                                    const void *v, const float *log_a, const float *b,
+                                    const int32_t *parent, const int32_t *node_offsets,
+                                    const float *S_root, void *out, float *U, float *snapshots,
+                                    void *workspace, size_t workspace_bytes, tv_stream_t stream);
+
+/* The baseline's commit: S_new = the snapshot of each sequence's accepted path's last node
+ * (S_root for an empty path), with the path checks of tv_tree_commit.  S_new must not be
+ * S_root.  snapshots as written by tv_snapshot_verify on the same tree. */
+TV_API tv_status tv_snapshot_commit(const tv_problem *p, const float *snapshots,
+                                    const float *S_root, const int32_t *node_offsets,
+                                    const int32_t *accepted_path, const int32_t *parent,
+                                    float *S_new, void *workspace, size_t workspace_bytes,
+                                    tv_stream_t stream);
+
 /* Diagnostic, with no counterpart on the pages: enqueue one small kernel whose bounded
  * wait on an mbarrier phase that never completes runs out.  It then records
  * TV_ERR_TIMEOUT in `workspace`, as a verify or commit CTA does after a wait that does not

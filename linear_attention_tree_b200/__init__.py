@@ -7,7 +7,9 @@ the accepted path's state from those pseudo-values.  Both are CUDA kernels behin
 ABI of ``include/tree_verify.h``; this package is the Python binding over it.
 """
 from .binding import (TreeVerifyError, get_status, lib, make_problem, new_workspace,
-                      tree_commit, tree_commit_verify, tree_meta, tree_verify, workspace_size)
+                      snapshot_commit, snapshot_verify, tree_commit, tree_commit_verify,
+                      tree_meta, tree_verify, workspace_size)
 
-__all__ = ["tree_verify", "tree_commit", "tree_commit_verify", "tree_meta", "get_status", "workspace_size",
+__all__ = ["tree_verify", "tree_commit", "tree_commit_verify", "snapshot_verify",
+           "snapshot_commit", "tree_meta", "get_status", "workspace_size",
            "new_workspace", "make_problem", "lib", "TreeVerifyError"]

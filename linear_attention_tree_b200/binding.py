@@ -10,6 +10,8 @@ Python name  -> C entry point
   tree_commit     tv_tree_commit
   tree_meta       tv_tree_meta
   tree_commit_verify tv_tree_commit_verify
+  snapshot_verify tv_snapshot_verify    (the per-node-snapshot baseline)
+  snapshot_commit tv_snapshot_commit
   workspace_size  tv_workspace_size
   get_status      tv_get_status
   selftest_timeout tv_selftest_timeout
@@ -31,7 +33,7 @@ MODE = {"gdn": 0, "scalar": 1}
 DTYPE = {torch.float32: 0, torch.bfloat16: 1}
 KERNEL = {"auto": 0, "tc": 1, "simt": 2}
 EXPORTS = ("tv_workspace_size", "tv_tree_verify", "tv_tree_commit", "tv_tree_meta",
-           "tv_tree_commit_verify",
+           "tv_tree_commit_verify", "tv_snapshot_verify", "tv_snapshot_commit",
            "tv_get_status", "tv_status_string", "tv_last_cuda_error", "tv_version",
            "tv_selftest_timeout")
 
@@ -73,6 +75,10 @@ def lib() -> ctypes.CDLL:
         L.tv_tree_meta.argtypes = [P] + [vp] * 7 + [ctypes.c_size_t, vp]
         L.tv_tree_commit_verify.argtypes = [P] + [vp] * 8 + [P] + [vp] * 10 + [ctypes.c_size_t, vp]
         L.tv_tree_commit_verify.restype = ctypes.c_int
+        L.tv_snapshot_verify.argtypes = [P] + [vp] * 12 + [ctypes.c_size_t, vp]
+        L.tv_snapshot_verify.restype = ctypes.c_int
+        L.tv_snapshot_commit.argtypes = [P] + [vp] * 7 + [ctypes.c_size_t, vp]
+        L.tv_snapshot_commit.restype = ctypes.c_int
         L.tv_tree_meta.restype = ctypes.c_int
         L.tv_get_status.argtypes = [vp, vp]
         L.tv_get_status.restype = ctypes.c_int
@@ -268,6 +274,69 @@ def tree_commit_verify(U_prev, k_prev, log_a_prev, node_offsets_prev, accepted_p
                                      ctypes.c_size_t(workspace.numel()), _stream(stream))
     _check(st, "tv_tree_commit_verify")
     return S_new, out, U
+
+
+def snapshot_verify(q, k, v, log_a, b, parent, node_offsets, S_root, *, max_nodes: int,
+                    mode: str = "gdn", snapshots=None, out=None, U=None, out_dtype=None,
+                    workspace=None, stream=None):
+    """The per-node-snapshot baseline; returns (out, U, snapshots [T][H][dv][dk] fp32)."""
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    B = node_offsets.shape[0] - 1
+    dev = q.device
+    out_dtype = out_dtype or q.dtype
+    if out is None:
+        out = torch.empty((T, H, dv), dtype=out_dtype, device=dev)
+    if U is None:
+        U = torch.empty((T, H, dv), dtype=torch.float32, device=dev)
+    if snapshots is None:
+        snapshots = torch.empty((T, H, dv, dk), dtype=torch.float32, device=dev)
+    prob = make_problem(B, H, dk, dv, T, max_nodes, 1, mode, q.dtype, out.dtype)
+    if workspace is None:
+        workspace = new_workspace(prob, dev)
+    fdt = torch.float32
+    args = [
+        _ptr(q, "q", (torch.float32, torch.bfloat16), (T, H, dk), dev),
+        _ptr(k, "k", q.dtype, (T, H, dk), dev), _ptr(v, "v", q.dtype, (T, H, dv), dev),
+        _ptr(log_a, "log_a", fdt, (T, H), dev), _ptr(b, "b", fdt, (T, H), dev),
+        _ptr(parent, "parent", torch.int32, (T,), dev),
+        _ptr(node_offsets, "node_offsets", torch.int32, (B + 1,), dev),
+        _ptr(S_root, "S_root", fdt, (B, H, dv, dk), dev),
+        _ptr(out, "out", (torch.float32, torch.bfloat16), (T, H, dv), dev),
+        _ptr(U, "U", fdt, (T, H, dv), dev),
+        _ptr(snapshots, "snapshots", fdt, (T, H, dv, dk), dev),
+        _ptr(workspace, "workspace", torch.uint8, None, dev),
+    ]
+    _check(lib().tv_snapshot_verify(ctypes.byref(prob), *args, ctypes.c_size_t(workspace.numel()),
+                                    _stream(stream)), "tv_snapshot_verify")
+    return out, U, snapshots
+
+
+def snapshot_commit(snapshots, S_root, node_offsets, accepted_path, *, max_nodes: int,
+                    parent=None, S_new=None, workspace=None, stream=None):
+    """The baseline's commit: S_new = the snapshot of each accepted path's last node."""
+    T, H, dv, dk = snapshots.shape
+    B = node_offsets.shape[0] - 1
+    dev = snapshots.device
+    if S_new is None:
+        S_new = torch.empty_like(S_root)
+    max_path = accepted_path.shape[1]
+    prob = make_problem(B, H, dk, dv, T, max_nodes, max_path)
+    if workspace is None:
+        workspace = new_workspace(prob, dev)
+    fdt = torch.float32
+    args = [
+        _ptr(snapshots, "snapshots", fdt, (T, H, dv, dk), dev),
+        _ptr(S_root, "S_root", fdt, (B, H, dv, dk), dev),
+        _ptr(node_offsets, "node_offsets", torch.int32, (B + 1,), dev),
+        _ptr(accepted_path, "accepted_path", torch.int32, (B, max_path), dev),
+        _ptr(parent, "parent", torch.int32, (T,), dev),
+        _ptr(S_new, "S_new", fdt, (B, H, dv, dk), dev),
+        _ptr(workspace, "workspace", torch.uint8, None, dev),
+    ]
+    _check(lib().tv_snapshot_commit(ctypes.byref(prob), *args, ctypes.c_size_t(workspace.numel()),
+                                    _stream(stream)), "tv_snapshot_commit")
+    return S_new
 
 
 def tree_meta(parent, node_offsets, log_a, *, max_nodes: int, workspace=None, stream=None):

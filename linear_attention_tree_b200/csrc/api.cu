@@ -230,6 +230,52 @@ tv_status tv_tree_meta(const tv_problem *p, const int32_t *parent,
   return from_cuda(launch_meta(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+tv_status tv_snapshot_verify(const tv_problem *p, const void *q, const void *k, const void *v,
+                             const float *log_a, const float *b, const int32_t *parent,
+                             const int32_t *node_offsets, const float *S_root, void *out,
+                             float *U, float *snapshots, void *workspace, size_t workspace_bytes,
+                             tv_stream_t stream) {
+  tv_status st = check_problem(p);
+  if (st != TV_OK) return st;
+  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(log_a) || !ptr_ok(parent) ||
+      !ptr_ok(node_offsets) || !ptr_ok(S_root) || !ptr_ok(out) || !ptr_ok(U) ||
+      !ptr_ok(snapshots) || !ptr_ok(workspace))
+    return TV_ERR_INVALID_ARG;
+  if (p->mode == TV_MODE_GDN ? !ptr_ok(b) : (b && !aligned16(b))) return TV_ERR_INVALID_ARG;
+  if (workspace_bytes < kWorkspaceBytes) return TV_ERR_INVALID_ARG;
+  if (p->B == 0) return TV_OK;
+  VerifyArgs a;
+  a.q = q; a.k = k; a.v = v; a.log_a = log_a; a.b = b; a.parent = parent;
+  a.node_offsets = node_offsets; a.S_root = S_root; a.out = out; a.U = U;
+  a.ws = static_cast<int *>(workspace);
+  a.B = p->B; a.H = p->H; a.dk = p->dk; a.dv = p->dv; a.T = p->total_nodes;
+  a.max_nodes = p->max_nodes;
+  return from_cuda(launch_snapshot_verify(a, snapshots, p->mode, p->in_dtype, p->out_dtype,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tv_status tv_snapshot_commit(const tv_problem *p, const float *snapshots, const float *S_root,
+                             const int32_t *node_offsets, const int32_t *accepted_path,
+                             const int32_t *parent, float *S_new, void *workspace,
+                             size_t workspace_bytes, tv_stream_t stream) {
+  tv_status st = check_problem(p);
+  if (st != TV_OK) return st;
+  if (p->max_path < 1) return TV_ERR_INVALID_ARG;
+  if (!ptr_ok(snapshots) || !ptr_ok(S_root) || !ptr_ok(node_offsets) ||
+      !ptr_ok(accepted_path) || !ptr_ok(S_new) || !ptr_ok(workspace))
+    return TV_ERR_INVALID_ARG;
+  if (parent && !aligned16(parent)) return TV_ERR_INVALID_ARG;
+  if (workspace_bytes < kWorkspaceBytes) return TV_ERR_INVALID_ARG;
+  if (S_new == S_root) return TV_ERR_INVALID_ARG;   // other sequences may still read S_root
+  if (p->B == 0) return TV_OK;
+  CommitArgs a = {};
+  a.S_root = S_root; a.node_offsets = node_offsets; a.accepted_path = accepted_path;
+  a.parent = parent; a.S_new = S_new; a.ws = static_cast<int *>(workspace);
+  a.B = p->B; a.H = p->H; a.dk = p->dk; a.dv = p->dv; a.T = p->total_nodes;
+  a.max_nodes = p->max_nodes; a.max_path = p->max_path;
+  return from_cuda(launch_snapshot_commit(a, snapshots, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 tv_status tv_selftest_timeout(void *workspace, size_t workspace_bytes, tv_stream_t stream) {
   if (!ptr_ok(workspace) || workspace_bytes < kWorkspaceBytes) return TV_ERR_INVALID_ARG;
   // a short poll budget: the point is the path taken when a wait runs out, not its length

@@ -91,5 +91,8 @@ cudaError_t launch_verify_tcw(const VerifyArgs &a, int mode, int out_dtype, cuda
 int commit_max_path_width();
 cudaError_t launch_commit(const CommitArgs &a, int in_dtype, cudaStream_t st);
 cudaError_t launch_meta(const MetaArgs &a, cudaStream_t st);
+cudaError_t launch_snapshot_verify(const VerifyArgs &a, float *snap, int mode, int in_dtype,
+                                   int out_dtype, cudaStream_t st);
+cudaError_t launch_snapshot_commit(const CommitArgs &a, const float *snap, cudaStream_t st);
 
 }  // namespace tv
