@@ -620,6 +620,56 @@ def other_workloads(args, L, dev, peak) -> dict:
     return res
 
 
+CASES = {
+    "verify3": (3, "verify"), "verify4": (4, "verify"), "verify5": (5, "verify"),
+    "commit3": (3, "commit"), "fused3": (3, "fused"), "snapshot3": (3, "snapshot"),
+}
+
+
+def run_case(args) -> int:
+    """A few launches of one operation on one named workload and nothing else (no timing,
+    no output): the command a profiler wraps.  Input set 0; the state is not updated."""
+    import torch
+    import linear_attention_tree_b200 as L
+    from linear_attention_tree_b200 import workloads as W
+    from linear_attention_tree_b200.tensors import to_device
+    idx, op = CASES[args.case]
+    w = W.config(idx, 0)
+    d = to_device(w, "cuda")
+    ws = L.new_workspace(L.make_problem(w.B, w.H, w.dk, w.dv, w.T, w.max_nodes, w.max_path))
+    out = torch.empty((w.T, w.H, w.dv), dtype=torch.float32, device="cuda")
+    U = torch.empty_like(out)
+    U2 = torch.empty_like(out)
+    S = d["S_root"].clone()
+    S_new = torch.empty_like(S)
+    L.tree_verify(d["q"], d["k"], d["v"], d["log_a"], d["b"], d["parent"], d["node_offsets"],
+                  S, max_nodes=w.max_nodes, out=out, U=U, workspace=ws, kernel=args.kernel)
+    snap = (torch.empty((w.T, w.H, w.dv, w.dk), dtype=torch.float32, device="cuda")
+            if op == "snapshot" else None)
+    for _ in range(args.launches):
+        if op == "verify":
+            L.tree_verify(d["q"], d["k"], d["v"], d["log_a"], d["b"], d["parent"],
+                          d["node_offsets"], S, max_nodes=w.max_nodes, out=out, U=U,
+                          workspace=ws, kernel=args.kernel)
+        elif op == "commit":
+            L.tree_commit(U, d["k"], d["log_a"], S, d["node_offsets"], d["accepted_path"],
+                          max_nodes=w.max_nodes, S_new=S_new, workspace=ws)
+        elif op == "fused":
+            L.tree_commit_verify(U, d["k"], d["log_a"], d["node_offsets"], d["accepted_path"],
+                                 S, d["q"], d["k"], d["v"], d["log_a"], d["b"], d["parent"],
+                                 d["node_offsets"], max_nodes_prev=w.max_nodes,
+                                 max_nodes=w.max_nodes, S_new=S_new, out=out, U=U2,
+                                 workspace=ws, kernel=args.kernel)
+        else:
+            L.snapshot_verify(d["q"], d["k"], d["v"], d["log_a"], d["b"], d["parent"],
+                              d["node_offsets"], S, max_nodes=w.max_nodes, snapshots=snap,
+                              out=out, U=U2, workspace=ws)
+    torch.cuda.synchronize()
+    if L.get_status(ws) != 0:
+        raise RuntimeError("device status after the case")
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -632,7 +682,14 @@ def main(argv=None):
                     help="skip the per-node-snapshot baseline (4.3 GB of snapshots)")
     ap.add_argument("--other-configs-off", action="store_true",
                     help="skip the per-launch timing of the ragged and wide-tree workloads")
+    ap.add_argument("--case", choices=sorted(CASES),
+                    help="only launch one operation --launches times on one workload (for a "
+                         "profiler): verifyN = tv_tree_verify on workload N, commit3, fused3 = "
+                         "tv_tree_commit_verify, snapshot3 = the per-node-snapshot baseline")
+    ap.add_argument("--launches", type=int, default=3)
     args = ap.parse_args(argv)
+    if args.case:
+        return run_case(args)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from linear_attention_tree_b200 import workloads as W
