@@ -38,7 +38,8 @@
  *   node_offsets[s] .. node_offsets[s+1]-1, and parent[] holds local indices in
  *   topological order (parent[i] < i), -1 meaning "child of S_root".  A first-level node
  *   has depth 1.
- * - Layouts:  q, k [T][H][dk];  v, U, out [T][H][dv];  log_a, b [T][H];  parent [T];
+ * - Layouts:  q, k [T][Hk][dk] (Hk = qk_heads, H by default);  v, U, out [T][H][dv];
+ *   log_a, b [T][H];  parent [T];
  *   node_offsets [B+1];  S_root, S_new [B][H][dv][dk] (row v, column k);
  *   accepted_path [B][max_path] (root-first local indices, -1 padded at the tail).
  * - Errors in the arguments (NULL pointers, misalignment, bad sizes, unsupported shapes)
@@ -98,8 +99,9 @@ typedef enum { TV_F32 = 0, TV_BF16 = 1 } tv_dtype;
  * TV_ERR_UNSUPPORTED. */
 typedef enum { TV_KERNEL_AUTO = 0, TV_KERNEL_TC = 1, TV_KERNEL_SIMT = 2 } tv_kernel;
 
-/* Problem description (all fields int32 so that the layout is fixed: 11 x 4 bytes).
- *   B, H         sequences and heads (B >= 0, H >= 1)
+/* Problem description (all fields int32 so that the layout is fixed: 13 x 4 bytes; a
+ * zero-filled struct leaves the last two fields at their defaults).
+ *   B, H         sequences and (value) heads (B >= 0, H >= 1)
  *   dk, dv       key and value width: multiples of 16 in [16, 128]
  *   total_nodes  T = node_offsets[B]
  *   max_nodes    upper bound on any sequence's node count, 1..256
@@ -108,6 +110,13 @@ typedef enum { TV_KERNEL_AUTO = 0, TV_KERNEL_TC = 1, TV_KERNEL_SIMT = 2 } tv_ker
  *   in_dtype     storage type of q, k, v (TV_F32 or TV_BF16)
  *   out_dtype    storage type of out (TV_F32, or TV_BF16 when in_dtype is TV_BF16)
  *   kernel       tv_kernel (verify only)
+ *   u_dtype      storage type of U (TV_F32, the default, or TV_BF16: half the bytes for the
+ *                pseudo-values written by verify and read by commit; U is rounded to nearest
+ *                even once it is final, so o is unaffected; not on the CUDA-core kernel, which
+ *                reads its own U back)
+ *   qk_heads     number of q / k heads Hk (0 = H): value head h reads q / k head
+ *                h / (H / Hk), as when several value heads share one q / k head; H must be a
+ *                multiple of Hk.  q and k are then [T][Hk][dk]
  * The tensor-core kernels need in_dtype = TV_BF16 and dk = dv = 128 (any max_nodes: one
  * kernel takes trees of up to 64 nodes, another wider ones; trees deeper than 16 nodes
  * in the wider kernel are verified on CUDA cores inside the same launch). */
@@ -115,6 +124,7 @@ typedef struct {
   int32_t B, H, dk, dv;
   int32_t total_nodes, max_nodes, max_path;
   int32_t mode, in_dtype, out_dtype, kernel;
+  int32_t u_dtype, qk_heads;
 } tv_problem;
 
 /* Bytes of device workspace the entry points need for problem p (0 if p is invalid).
@@ -122,7 +132,7 @@ typedef struct {
 TV_API size_t tv_workspace_size(const tv_problem *p);
 
 /* Verify every node of every tree in one call.
- *   q, k      [T][H][dk] in_dtype          (device, read)
+ *   q, k      [T][Hk][dk] in_dtype         (device, read)
  *   v         [T][H][dv] in_dtype          (device, read)
  *   log_a     [T][H] fp32, log of the decay (device, read)
  *   b         [T][H] fp32 write strength   (device, read; may be NULL in scalar mode)
@@ -131,7 +141,7 @@ TV_API size_t tv_workspace_size(const tv_problem *p);
  *   S_root    [B][H][dv][dk] fp32          (device, read only: verify has no side effect
  *                                            on the state)
  *   out       [T][H][dv] out_dtype, o_n = S_n q_n                (device, written)
- *   U         [T][H][dv] fp32 pseudo-values u_n (scalar: v_n)    (device, written)
+ *   U         [T][H][dv] u_dtype pseudo-values u_n (scalar: v_n) (device, written)
  * out and U must not overlap any input.  Bit-for-bit deterministic run to run. */
 TV_API tv_status tv_tree_verify(const tv_problem *p, const void *q, const void *k, const void *v,
                          const float *log_a, const float *b, const int32_t *parent,
@@ -142,8 +152,8 @@ TV_API tv_status tv_tree_verify(const tv_problem *p, const void *q, const void *
 /* Rebuild the accepted state of every sequence from the pseudo-values:
  *   S_new = exp(c_m) S_root + sum_{j<=m} exp(c_m - c_j) u_{p_j} k_{p_j}^T,
  *   c_j = sum_{l<=j} log_a_{p_l}, along accepted_path p_1..p_m (root first).
- *   U          [T][H][dv] fp32 from tv_tree_verify on the same S_root (device, read)
- *   k          [T][H][dk] in_dtype          (device, read)
+ *   U          [T][H][dv] u_dtype from tv_tree_verify on the same S_root (device, read)
+ *   k          [T][Hk][dk] in_dtype         (device, read)
  *   log_a      [T][H] fp32                  (device, read)
  *   S_root     [B][H][dv][dk] fp32          (device, read)
  *   node_offsets [B+1] int32                (device, read)

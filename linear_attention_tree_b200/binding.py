@@ -50,7 +50,7 @@ class TreeVerifyError(RuntimeError):
 class Problem(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("B", "H", "dk", "dv", "total_nodes", "max_nodes", "max_path", "mode",
-                 "in_dtype", "out_dtype", "kernel")]
+                 "in_dtype", "out_dtype", "kernel", "u_dtype", "qk_heads")]
 
 
 _lib = None
@@ -99,10 +99,13 @@ def status_string(status: int) -> str:
 
 
 def make_problem(B, H, dk, dv, total_nodes, max_nodes, max_path=1, mode="gdn",
-                 in_dtype=torch.bfloat16, out_dtype=None, kernel="auto") -> Problem:
+                 in_dtype=torch.bfloat16, out_dtype=None, kernel="auto",
+                 u_dtype=torch.float32, qk_heads=0) -> Problem:
+    """``qk_heads``: number of q / k heads (0 = H); ``u_dtype``: storage type of U."""
     return Problem(int(B), int(H), int(dk), int(dv), int(total_nodes), int(max_nodes),
                    int(max_path), MODE[mode], DTYPE[in_dtype],
-                   DTYPE[out_dtype if out_dtype is not None else in_dtype], KERNEL[kernel])
+                   DTYPE[out_dtype if out_dtype is not None else in_dtype], KERNEL[kernel],
+                   DTYPE[u_dtype], int(qk_heads))
 
 
 def workspace_size(problem: Problem) -> int:
@@ -145,30 +148,33 @@ def _check(status: int, what: str):
 
 def tree_verify(q, k, v, log_a, b, parent, node_offsets, S_root, *, max_nodes: int,
                 mode: str = "gdn", out=None, U=None, out_dtype=None, workspace=None,
-                kernel: str = "auto", stream=None):
+                kernel: str = "auto", u_dtype=None, stream=None):
     """Verify every node of every draft tree; returns (out, U).
 
-    q, k [T][H][dk]; v [T][H][dv] (fp32 or bf16); log_a, b [T][H] fp32 (b may be None in
-    scalar mode); parent [T], node_offsets [B+1] int32; S_root [B][H][dv][dk] fp32.
-    out [T][H][dv] (out_dtype, default the input dtype) and U [T][H][dv] fp32 are allocated
-    when not given.  ``max_nodes`` bounds every sequence's node count (<= 256).
+    q, k [T][Hk][dk] (Hk q / k heads shared by H / Hk value heads each, Hk = H by default);
+    v [T][H][dv] (fp32 or bf16); log_a, b [T][H] fp32 (b may be None in scalar mode);
+    parent [T], node_offsets [B+1] int32; S_root [B][H][dv][dk] fp32.  out [T][H][dv]
+    (out_dtype, default the input dtype) and U [T][H][dv] (u_dtype, default fp32, or the
+    dtype of the U given) are allocated when not given.  ``max_nodes`` bounds every
+    sequence's node count (<= 256).
     """
-    T, H, dk = q.shape
-    dv = v.shape[2]
+    T, Hk, dk = q.shape
+    H, dv = v.shape[1], v.shape[2]
     B = node_offsets.shape[0] - 1
     dev = q.device
     out_dtype = out_dtype or q.dtype
     if out is None:
         out = torch.empty((T, H, dv), dtype=out_dtype, device=dev)
     if U is None:
-        U = torch.empty((T, H, dv), dtype=torch.float32, device=dev)
-    prob = make_problem(B, H, dk, dv, T, max_nodes, 1, mode, q.dtype, out.dtype, kernel)
+        U = torch.empty((T, H, dv), dtype=u_dtype or torch.float32, device=dev)
+    prob = make_problem(B, H, dk, dv, T, max_nodes, 1, mode, q.dtype, out.dtype, kernel,
+                        U.dtype, 0 if Hk == H else Hk)
     if workspace is None:
         workspace = new_workspace(prob, dev)
     fdt = torch.float32
     args = [
-        _ptr(q, "q", (torch.float32, torch.bfloat16), (T, H, dk), dev),
-        _ptr(k, "k", q.dtype, (T, H, dk), dev),
+        _ptr(q, "q", (torch.float32, torch.bfloat16), (T, Hk, dk), dev),
+        _ptr(k, "k", q.dtype, (T, Hk, dk), dev),
         _ptr(v, "v", q.dtype, (T, H, dv), dev),
         _ptr(log_a, "log_a", fdt, (T, H), dev),
         _ptr(b, "b", fdt, (T, H), dev),
@@ -176,7 +182,7 @@ def tree_verify(q, k, v, log_a, b, parent, node_offsets, S_root, *, max_nodes: i
         _ptr(node_offsets, "node_offsets", torch.int32, (B + 1,), dev),
         _ptr(S_root, "S_root", fdt, (B, H, dv, dk), dev),
         _ptr(out, "out", (torch.float32, torch.bfloat16), (T, H, dv), dev),
-        _ptr(U, "U", fdt, (T, H, dv), dev),
+        _ptr(U, "U", (torch.float32, torch.bfloat16), (T, H, dv), dev),
         _ptr(workspace, "workspace", torch.uint8, None, dev),
     ]
     st = lib().tv_tree_verify(ctypes.byref(prob), *args, ctypes.c_size_t(workspace.numel()),
@@ -193,19 +199,20 @@ def tree_commit(U, k, log_a, S_root, node_offsets, accepted_path, *, max_nodes: 
     int32, root-first, -1 padded.  With ``parent`` every path is checked against its tree.
     """
     T, H, dv = U.shape
-    dk = k.shape[2]
+    Hk, dk = k.shape[1], k.shape[2]
     B = node_offsets.shape[0] - 1
     dev = U.device
     if S_new is None:
         S_new = torch.empty_like(S_root)
     max_path = accepted_path.shape[1] if accepted_path.dim() == 2 else 0
-    prob = make_problem(B, H, dk, dv, T, max_nodes, max_path, "gdn", k.dtype, k.dtype)
+    prob = make_problem(B, H, dk, dv, T, max_nodes, max_path, "gdn", k.dtype, k.dtype,
+                        u_dtype=U.dtype, qk_heads=0 if Hk == H else Hk)
     if workspace is None:
         workspace = new_workspace(prob, dev)
     fdt = torch.float32
     args = [
-        _ptr(U, "U", fdt, (T, H, dv), dev),
-        _ptr(k, "k", (torch.float32, torch.bfloat16), (T, H, dk), dev),
+        _ptr(U, "U", (torch.float32, torch.bfloat16), (T, H, dv), dev),
+        _ptr(k, "k", (torch.float32, torch.bfloat16), (T, Hk, dk), dev),
         _ptr(log_a, "log_a", fdt, (T, H), dev),
         _ptr(S_root, "S_root", fdt, (B, H, dv, dk), dev),
         _ptr(node_offsets, "node_offsets", torch.int32, (B + 1,), dev),
@@ -230,7 +237,7 @@ def tree_commit_verify(U_prev, k_prev, log_a_prev, node_offsets_prev, accepted_p
     ``U_prev``.  Argument meanings as in `tree_commit` (previous tree) and `tree_verify`
     (next tree)."""
     Tp, H, dv = U_prev.shape
-    dk = k_prev.shape[2]
+    Hk, dk = k_prev.shape[1], k_prev.shape[2]
     B = node_offsets.shape[0] - 1
     T = q.shape[0]
     dev = q.device
@@ -240,17 +247,19 @@ def tree_commit_verify(U_prev, k_prev, log_a_prev, node_offsets_prev, accepted_p
     if out is None:
         out = torch.empty((T, H, dv), dtype=out_dtype, device=dev)
     if U is None:
-        U = torch.empty((T, H, dv), dtype=torch.float32, device=dev)
+        U = torch.empty((T, H, dv), dtype=U_prev.dtype, device=dev)
     max_path = accepted_path.shape[1]
+    qkh = 0 if Hk == H else Hk
     prev = make_problem(B, H, dk, dv, Tp, max_nodes_prev, max_path, mode, k_prev.dtype,
-                        k_prev.dtype)
-    nxt = make_problem(B, H, dk, dv, T, max_nodes, 1, mode, q.dtype, out.dtype, kernel)
+                        k_prev.dtype, u_dtype=U_prev.dtype, qk_heads=qkh)
+    nxt = make_problem(B, H, dk, dv, T, max_nodes, 1, mode, q.dtype, out.dtype, kernel,
+                       U.dtype, qkh)
     if workspace is None:
         workspace = new_workspace(nxt, dev)
     fdt = torch.float32
     args = [
-        _ptr(U_prev, "U_prev", fdt, (Tp, H, dv), dev),
-        _ptr(k_prev, "k_prev", (torch.float32, torch.bfloat16), (Tp, H, dk), dev),
+        _ptr(U_prev, "U_prev", (torch.float32, torch.bfloat16), (Tp, H, dv), dev),
+        _ptr(k_prev, "k_prev", (torch.float32, torch.bfloat16), (Tp, Hk, dk), dev),
         _ptr(log_a_prev, "log_a_prev", fdt, (Tp, H), dev),
         _ptr(node_offsets_prev, "node_offsets_prev", torch.int32, (B + 1,), dev),
         _ptr(accepted_path, "accepted_path", torch.int32, (B, max_path), dev),
@@ -259,15 +268,15 @@ def tree_commit_verify(U_prev, k_prev, log_a_prev, node_offsets_prev, accepted_p
         _ptr(S_new, "S_new", fdt, (B, H, dv, dk), dev),
     ]
     args2 = [
-        _ptr(q, "q", (torch.float32, torch.bfloat16), (T, H, dk), dev),
-        _ptr(k, "k", q.dtype, (T, H, dk), dev),
+        _ptr(q, "q", (torch.float32, torch.bfloat16), (T, Hk, dk), dev),
+        _ptr(k, "k", q.dtype, (T, Hk, dk), dev),
         _ptr(v, "v", q.dtype, (T, H, dv), dev),
         _ptr(log_a, "log_a", fdt, (T, H), dev),
         _ptr(b, "b", fdt, (T, H), dev),
         _ptr(parent, "parent", torch.int32, (T,), dev),
         _ptr(node_offsets, "node_offsets", torch.int32, (B + 1,), dev),
         _ptr(out, "out", (torch.float32, torch.bfloat16), (T, H, dv), dev),
-        _ptr(U, "U", fdt, (T, H, dv), dev),
+        _ptr(U, "U", (torch.float32, torch.bfloat16), (T, H, dv), dev),
         _ptr(workspace, "workspace", torch.uint8, None, dev),
     ]
     st = lib().tv_tree_commit_verify(ctypes.byref(prev), *args, ctypes.byref(nxt), *args2,
@@ -280,8 +289,8 @@ def snapshot_verify(q, k, v, log_a, b, parent, node_offsets, S_root, *, max_node
                     mode: str = "gdn", snapshots=None, out=None, U=None, out_dtype=None,
                     workspace=None, stream=None):
     """The per-node-snapshot baseline; returns (out, U, snapshots [T][H][dv][dk] fp32)."""
-    T, H, dk = q.shape
-    dv = v.shape[2]
+    T, Hk, dk = q.shape
+    H, dv = v.shape[1], v.shape[2]
     B = node_offsets.shape[0] - 1
     dev = q.device
     out_dtype = out_dtype or q.dtype
@@ -291,19 +300,20 @@ def snapshot_verify(q, k, v, log_a, b, parent, node_offsets, S_root, *, max_node
         U = torch.empty((T, H, dv), dtype=torch.float32, device=dev)
     if snapshots is None:
         snapshots = torch.empty((T, H, dv, dk), dtype=torch.float32, device=dev)
-    prob = make_problem(B, H, dk, dv, T, max_nodes, 1, mode, q.dtype, out.dtype)
+    prob = make_problem(B, H, dk, dv, T, max_nodes, 1, mode, q.dtype, out.dtype,
+                        u_dtype=U.dtype, qk_heads=0 if Hk == H else Hk)
     if workspace is None:
         workspace = new_workspace(prob, dev)
     fdt = torch.float32
     args = [
-        _ptr(q, "q", (torch.float32, torch.bfloat16), (T, H, dk), dev),
-        _ptr(k, "k", q.dtype, (T, H, dk), dev), _ptr(v, "v", q.dtype, (T, H, dv), dev),
+        _ptr(q, "q", (torch.float32, torch.bfloat16), (T, Hk, dk), dev),
+        _ptr(k, "k", q.dtype, (T, Hk, dk), dev), _ptr(v, "v", q.dtype, (T, H, dv), dev),
         _ptr(log_a, "log_a", fdt, (T, H), dev), _ptr(b, "b", fdt, (T, H), dev),
         _ptr(parent, "parent", torch.int32, (T,), dev),
         _ptr(node_offsets, "node_offsets", torch.int32, (B + 1,), dev),
         _ptr(S_root, "S_root", fdt, (B, H, dv, dk), dev),
         _ptr(out, "out", (torch.float32, torch.bfloat16), (T, H, dv), dev),
-        _ptr(U, "U", fdt, (T, H, dv), dev),
+        _ptr(U, "U", (torch.float32, torch.bfloat16), (T, H, dv), dev),
         _ptr(snapshots, "snapshots", fdt, (T, H, dv, dk), dev),
         _ptr(workspace, "workspace", torch.uint8, None, dev),
     ]

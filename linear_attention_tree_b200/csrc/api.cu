@@ -21,6 +21,9 @@ tv_status check_problem(const tv_problem *p) {
   if (p->out_dtype != TV_F32 && p->out_dtype != TV_BF16) return TV_ERR_INVALID_ARG;
   if (p->kernel < TV_KERNEL_AUTO || p->kernel > TV_KERNEL_SIMT) return TV_ERR_INVALID_ARG;
   if (p->dk < 1 || p->dv < 1) return TV_ERR_INVALID_ARG;
+  if (p->u_dtype != TV_F32 && p->u_dtype != TV_BF16) return TV_ERR_INVALID_ARG;
+  if (p->qk_heads < 0 || p->qk_heads > p->H || (p->qk_heads && p->H % p->qk_heads))
+    return TV_ERR_INVALID_ARG;
   if (p->max_nodes > kMaxNodes) return TV_ERR_UNSUPPORTED;
   if (p->dk % 16 || p->dv % 16 || p->dk > 128 || p->dv > 128) return TV_ERR_UNSUPPORTED;
   if (p->in_dtype == TV_F32 && p->out_dtype == TV_BF16) return TV_ERR_UNSUPPORTED;
@@ -32,6 +35,8 @@ tv_status check_problem(const tv_problem *p) {
 }
 
 bool ptr_ok(const void *ptr) { return ptr && aligned16(ptr); }
+
+int qk_heads_of(const tv_problem *p) { return p->qk_heads ? p->qk_heads : p->H; }
 
 bool tc_supports(const tv_problem *p) {
   return p->in_dtype == TV_BF16 && p->dk == 128 && p->dv == 128 &&
@@ -54,7 +59,7 @@ tv_status record_cuda_error(cudaError_t e) { return from_cuda(e); }
 
 extern "C" {
 
-int32_t tv_version(void) { return (1 << 16) | 0; }
+int32_t tv_version(void) { return (2 << 16) | 0; }   // 2: tv_problem gained u_dtype and qk_heads
 
 const char *tv_last_cuda_error(void) {
   if (g_last_cuda == cudaSuccess) return "";
@@ -101,13 +106,15 @@ tv_status tv_tree_verify(const tv_problem *p, const void *q, const void *k, cons
   } else {
     use_tc = p->kernel == TV_KERNEL_AUTO && tc_supports(p);
   }
+  // the CUDA-core kernel reads U back as it goes: it keeps it in fp32
+  if (!use_tc && p->u_dtype == TV_BF16) return TV_ERR_UNSUPPORTED;
   if (p->B == 0) return TV_OK;
   VerifyArgs a;
   a.q = q; a.k = k; a.v = v; a.log_a = log_a; a.b = b; a.parent = parent;
   a.node_offsets = node_offsets; a.S_root = S_root; a.out = out; a.U = U;
   a.ws = static_cast<int *>(workspace);
   a.B = p->B; a.H = p->H; a.dk = p->dk; a.dv = p->dv; a.T = p->total_nodes;
-  a.max_nodes = p->max_nodes;
+  a.max_nodes = p->max_nodes; a.Hk = qk_heads_of(p); a.u_bf16 = p->u_dtype == TV_BF16;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (use_tc)   // trees of up to 64 nodes, and wider trees, have one tensor-core kernel each
     return from_cuda(p->max_nodes <= verify_tc_max_nodes()
@@ -141,6 +148,7 @@ tv_status tv_tree_commit(const tv_problem *p, const float *U, const void *k,
   a.ws = static_cast<int *>(workspace);
   a.B = p->B; a.H = p->H; a.dk = p->dk; a.dv = p->dv; a.T = p->total_nodes;
   a.max_nodes = p->max_nodes; a.max_path = p->max_path;
+  a.Hk = qk_heads_of(p); a.u_bf16 = p->u_dtype == TV_BF16;
   return from_cuda(launch_commit(a, p->in_dtype, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -155,7 +163,8 @@ tv_status tv_tree_commit_verify(const tv_problem *prev, const float *U_prev, con
   tv_status st = check_problem(prev);
   if (st == TV_OK) st = check_problem(next);
   if (st != TV_OK) return st;
-  if (prev->B != next->B || prev->H != next->H || prev->dk != next->dk || prev->dv != next->dv)
+  if (prev->B != next->B || prev->H != next->H || prev->dk != next->dk || prev->dv != next->dv ||
+      qk_heads_of(prev) != qk_heads_of(next))
     return TV_ERR_INVALID_ARG;
   if (prev->max_path < 1) return TV_ERR_INVALID_ARG;
   if (prev->max_path > commit_max_path_width()) return TV_ERR_UNSUPPORTED;
@@ -171,20 +180,24 @@ tv_status tv_tree_commit_verify(const tv_problem *prev, const float *U_prev, con
   const char *a0 = reinterpret_cast<const char *>(S_root), *b0 = reinterpret_cast<const char *>(S_new);
   if (a0 != b0 && a0 < b0 + state_bytes && b0 < a0 + state_bytes) return TV_ERR_INVALID_ARG;
   // the new pseudo-values must not overwrite the previous ones while they are read
-  const size_t u_prev_bytes = (size_t)prev->total_nodes * prev->H * prev->dv * sizeof(float);
-  const size_t u_bytes = (size_t)next->total_nodes * next->H * next->dv * sizeof(float);
+  const size_t u_prev_bytes = (size_t)prev->total_nodes * prev->H * prev->dv *
+                              (prev->u_dtype == TV_BF16 ? 2 : 4);
+  const size_t u_bytes = (size_t)next->total_nodes * next->H * next->dv *
+                         (next->u_dtype == TV_BF16 ? 2 : 4);
   const char *c0 = reinterpret_cast<const char *>(U_prev), *d0 = reinterpret_cast<const char *>(U);
   if (u_prev_bytes && u_bytes && c0 < d0 + u_bytes && d0 < c0 + u_prev_bytes) return TV_ERR_INVALID_ARG;
   if (next->kernel == TV_KERNEL_TC && !tc_supports(next)) return TV_ERR_UNSUPPORTED;
+  const bool next_tc = next->kernel != TV_KERNEL_SIMT && tc_supports(next);
+  if (!next_tc && next->u_dtype == TV_BF16) return TV_ERR_UNSUPPORTED;
   if (next->B == 0) return TV_OK;
   VerifyArgs a;
   a.q = q; a.k = k; a.v = v; a.log_a = log_a; a.b = b; a.parent = parent;
   a.node_offsets = node_offsets; a.S_root = S_root; a.out = out; a.U = U;
   a.ws = static_cast<int *>(workspace);
   a.B = next->B; a.H = next->H; a.dk = next->dk; a.dv = next->dv; a.T = next->total_nodes;
-  a.max_nodes = next->max_nodes;
+  a.max_nodes = next->max_nodes; a.Hk = qk_heads_of(next); a.u_bf16 = next->u_dtype == TV_BF16;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const bool fused = next->kernel != TV_KERNEL_SIMT && tc_supports(next) &&
+  const bool fused = next_tc &&
                      next->max_nodes <= verify_tc_max_nodes() && prev->in_dtype == TV_BF16 &&
                      prev->max_path <= fused_max_path();
   if (fused) {
@@ -192,6 +205,7 @@ tv_status tv_tree_commit_verify(const tv_problem *prev, const float *U_prev, con
     f.U = U_prev; f.k = k_prev; f.log_a = log_a_prev; f.node_offsets = node_offsets_prev;
     f.accepted_path = accepted_path; f.parent = parent_prev; f.S_new = S_new;
     f.T = prev->total_nodes; f.max_nodes = prev->max_nodes; f.max_path = prev->max_path;
+    f.u_bf16 = prev->u_dtype == TV_BF16;
     return from_cuda(launch_commit_verify_tc(a, f, next->mode, next->out_dtype, s));
   }
   // otherwise the commit, then the verify on its result: two launches, same results
@@ -201,10 +215,11 @@ tv_status tv_tree_commit_verify(const tv_problem *prev, const float *U_prev, con
   c.S_new = S_new; c.ws = a.ws;
   c.B = prev->B; c.H = prev->H; c.dk = prev->dk; c.dv = prev->dv; c.T = prev->total_nodes;
   c.max_nodes = prev->max_nodes; c.max_path = prev->max_path;
+  c.Hk = qk_heads_of(prev); c.u_bf16 = prev->u_dtype == TV_BF16;
   st = from_cuda(launch_commit(c, prev->in_dtype, s));
   if (st != TV_OK) return st;
   a.S_root = S_new;
-  if (next->kernel != TV_KERNEL_SIMT && tc_supports(next))
+  if (next_tc)
     return from_cuda(next->max_nodes <= verify_tc_max_nodes()
                          ? launch_verify_tc(a, next->mode, next->out_dtype, s)
                          : launch_verify_tcw(a, next->mode, next->out_dtype, s));
@@ -249,7 +264,7 @@ tv_status tv_snapshot_verify(const tv_problem *p, const void *q, const void *k, 
   a.node_offsets = node_offsets; a.S_root = S_root; a.out = out; a.U = U;
   a.ws = static_cast<int *>(workspace);
   a.B = p->B; a.H = p->H; a.dk = p->dk; a.dv = p->dv; a.T = p->total_nodes;
-  a.max_nodes = p->max_nodes;
+  a.max_nodes = p->max_nodes; a.Hk = qk_heads_of(p); a.u_bf16 = p->u_dtype == TV_BF16;
   return from_cuda(launch_snapshot_verify(a, snapshots, p->mode, p->in_dtype, p->out_dtype,
                                           reinterpret_cast<cudaStream_t>(stream)));
 }

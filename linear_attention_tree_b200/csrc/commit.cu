@@ -53,6 +53,7 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(CommitArgs a) {
   const int H = a.H, dk = a.dk, dv = a.dv;
   const int slices = (dv + kRows - 1) / kRows;
   const int s = blockIdx.x / (H * slices), h = (blockIdx.x / slices) % H;
+  const int Hk = a.Hk, kh = qk_head(h, H, Hk);
   const int r0 = (blockIdx.x % slices) * kRows;           // first state row of the slice
   const int rows = min(kRows, dv - r0);
   const Tk *k = static_cast<const Tk *>(a.k);
@@ -116,9 +117,9 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(CommitArgs a) {
   const int cnt0 = min(kChunk, m);
   for (int e = tid; e < cnt0 * 128; e += kThreads) {
     const int j = e >> 7, x = e & 127;
-    const size_t node = (size_t)(lo + sm.prow[j]) * H + h;
-    if (x < rows) sm.cu[j][x] = a.U[node * dv + r0 + x];
-    if (x < dk) sm.kk[j][x] = to_f32(k[node * dk + x]);
+    const int row = lo + sm.prow[j];
+    if (x < rows) sm.cu[j][x] = load_u(a.U, ((size_t)row * H + h) * dv + r0 + x, a.u_bf16);
+    if (x < dk) sm.kk[j][x] = to_f32(k[((size_t)row * Hk + kh) * dk + x]);
   }
   if (__syncthreads_or(chain_bad)) {
     if (tid == 0 && r0 == 0) set_status(a.ws, TV_ERR_BAD_PATH, s);
@@ -148,9 +149,10 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(CommitArgs a) {
       __syncthreads();
       for (int e = tid; e < cnt * 128; e += kThreads) {
         const int j = e >> 7, x = e & 127;
-        const size_t node = (size_t)(lo + sm.prow[j0 + j]) * H + h;
-        if (x < rows) sm.cu[j][x] = sm.e[j0 + j] * a.U[node * dv + r0 + x];
-        if (x < dk) sm.kk[j][x] = to_f32(k[node * dk + x]);
+        const int row = lo + sm.prow[j0 + j];
+        if (x < rows)
+          sm.cu[j][x] = sm.e[j0 + j] * load_u(a.U, ((size_t)row * H + h) * dv + r0 + x, a.u_bf16);
+        if (x < dk) sm.kk[j][x] = to_f32(k[((size_t)row * Hk + kh) * dk + x]);
       }
       __syncthreads();
     }
@@ -328,16 +330,22 @@ __device__ void gather_path(const CommitArgs &a, int it, PathBuf &pb, const Path
 // in pb.prow), decay weights, and the u and k rows of the first kPathRows entries.
 template <typename Tk>
 __device__ void gather_rows(const CommitArgs &a, int it, PathBuf &pb, int m, int lo, int lane) {
-  const int H = a.H, h = it % H;
+  const int H = a.H, h = it % H, kh = qk_head(h, H, a.Hk);
   // log_a and the parent chain of every path entry; the u and k rows of the first
-  // kPathRows entries go straight into the buffer by asynchronous copies
+  // kPathRows entries go straight into the buffer by asynchronous copies (bf16 u rows land
+  // in the first half of their row and are widened when they are scaled)
   const Tk *k = static_cast<const Tk *>(a.k);
   Tk *kk = reinterpret_cast<Tk *>(&pb.kk[0][0]);
   const int staged = min(m, kPathRows);
   for (int j = 0; j < staged; ++j) {
-    const size_t node = (size_t)(lo + pb.prow[j]) * H + h;
-    cp_async16(&pb.cu[j][4 * lane], a.U + node * 128 + 4 * lane);
-    cp_async_k(kk + j * 128 + 4 * lane, k + node * 128 + 4 * lane);
+    const int row = lo + pb.prow[j];
+    const size_t node = (size_t)row * H + h;
+    if (a.u_bf16)
+      cp_async8(reinterpret_cast<__nv_bfloat16 *>(&pb.cu[j][0]) + 4 * lane,
+                static_cast<const __nv_bfloat16 *>(a.U) + node * 128 + 4 * lane);
+    else
+      cp_async16(&pb.cu[j][4 * lane], static_cast<const float *>(a.U) + node * 128 + 4 * lane);
+    cp_async_k(kk + j * 128 + 4 * lane, k + ((size_t)row * a.Hk + kh) * 128 + 4 * lane);
   }
   int chain_bad = 0;
   for (int t = lane; t < m; t += 32) {
@@ -372,7 +380,15 @@ __device__ void gather_rows(const CommitArgs &a, int it, PathBuf &pb, int m, int
       // each lane scales the 4 columns it copied
       float4 *c4 = reinterpret_cast<float4 *>(&pb.cu[j][4 * lane]);
       const float e = pb.e[j];
-      const float4 u = *c4;
+      float4 u;
+      if (a.u_bf16) {
+        const uint2 r = reinterpret_cast<const uint2 *>(&pb.cu[j][0])[lane];
+        u = make_float4(__uint_as_float(r.x << 16), __uint_as_float(r.x & 0xFFFF0000u),
+                        __uint_as_float(r.y << 16), __uint_as_float(r.y & 0xFFFF0000u));
+        __syncwarp();   // every lane has read its bf16 values before the row is widened
+      } else {
+        u = *c4;
+      }
       *c4 = make_float4(e * u.x, e * u.y, e * u.z, e * u.w);
     }
   __syncwarp();
@@ -499,14 +515,15 @@ __global__ void __launch_bounds__(kSThreads, 1) commit_stream_kernel(CommitArgs 
           }
         }
         // path entries past the staged ones come straight from HBM
-        const int h = it % a.H;
+        const int h = it % a.H, kh = qk_head(h, a.H, a.Hk);
         for (int j = staged; j < m; ++j) {
-          const size_t node = (size_t)(pb.lo + pb.prow[j]) * a.H + h;
-          const float4 kv = load_k4(k, node * 128 + col);
+          const int row = pb.lo + pb.prow[j];
+          const size_t node = (size_t)row * a.H + h;
+          const float4 kv = load_k4(k, ((size_t)row * a.Hk + kh) * 128 + col);
           const float e = pb.e[j];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float cu = e * a.U[node * 128 + rb + 16 * i];
+            const float cu = e * load_u(a.U, node * 128 + rb + 16 * i, a.u_bf16);
             acc[i].x = fmaf(cu, kv.x, acc[i].x);
             acc[i].y = fmaf(cu, kv.y, acc[i].y);
             acc[i].z = fmaf(cu, kv.z, acc[i].z);

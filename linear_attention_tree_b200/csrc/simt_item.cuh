@@ -54,6 +54,7 @@ __device__ void simt_item(const VerifyArgs &a, int s, int h, unsigned char *smem
   float *S = reinterpret_cast<float *>(smem_raw + sizeof(SimtSmem));
   const int tid = threadIdx.x;
   const int H = a.H, dk = a.dk, dv = a.dv, ldS = a.dk + 1;
+  const int Hk = a.Hk, kh = qk_head(h, H, Hk);
   const Tin *q = static_cast<const Tin *>(a.q);
   const Tin *k = static_cast<const Tin *>(a.k);
   const Tin *vv = static_cast<const Tin *>(a.v);
@@ -106,7 +107,7 @@ __device__ void simt_item(const VerifyArgs &a, int s, int h, unsigned char *smem
 
   const int warp = tid >> 5, lane = tid & 31;
   for (int n = 0; n < n_nodes; ++n) {
-    const size_t rowq = ((size_t)(lo + n) * H + h) * dk;
+    const size_t rowq = ((size_t)(lo + n) * Hk + kh) * dk;
     for (int j = tid; j < dk; j += kNT) {
       sm.qn[j] = to_f32(q[rowq + j]);
       sm.kn[j] = to_f32(k[rowq + j]);
@@ -130,7 +131,7 @@ __device__ void simt_item(const VerifyArgs &a, int s, int h, unsigned char *smem
     // path Gram terms, one warp per path entry
     for (int e = warp; e < plen; e += kNT / 32) {
       const int i = sm.plist[e];
-      const size_t rowk = ((size_t)(lo + i) * H + h) * dk;
+      const size_t rowk = ((size_t)(lo + i) * Hk + kh) * dk;
       float gq = 0.f, gk = 0.f;
       for (int j = lane; j < dk; j += 32) {
         const float ki = to_f32(k[rowk + j]);
@@ -164,15 +165,15 @@ __device__ void simt_item(const VerifyArgs &a, int s, int h, unsigned char *smem
       if (kGdn) {
         u = bn * (vn - gam * sk);
         for (int e = 0; e < plen - 1; ++e)
-          u = fmaf(-sm.ck[e], a.U[((size_t)(lo + sm.plist[e]) * H + h) * dv + col], u);
+          u = fmaf(-sm.ck[e], load_u(a.U, ((size_t)(lo + sm.plist[e]) * H + h) * dv + col, a.u_bf16), u);
       } else {
         u = vn;
       }
       float o = gam * sq;
       for (int e = 0; e < plen - 1; ++e)
-        o = fmaf(sm.cq[e], a.U[((size_t)(lo + sm.plist[e]) * H + h) * dv + col], o);
+        o = fmaf(sm.cq[e], load_u(a.U, ((size_t)(lo + sm.plist[e]) * H + h) * dv + col, a.u_bf16), o);
       o = fmaf(sm.cq[plen - 1], u, o);
-      a.U[rowv + col] = u;
+      store_u(a.U, rowv + col, u, a.u_bf16);
       out[rowv + col] = from_f32<Tout>(o);
     }
     __syncthreads();

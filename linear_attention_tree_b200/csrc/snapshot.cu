@@ -26,7 +26,7 @@ __global__ void __launch_bounds__(kThreads) snapshot_verify_kernel(VerifyArgs a,
   __shared__ int par, bad;
   const int t = threadIdx.x;
   const int s = blockIdx.x / a.H, h = blockIdx.x % a.H;
-  const int H = a.H, dk = a.dk, dv = a.dv;
+  const int H = a.H, dk = a.dk, dv = a.dv, kh = qk_head(h, H, a.Hk);
   const int lo = a.node_offsets[s], hi = a.node_offsets[s + 1];
   if (lo < 0 || hi < lo || hi > a.T || hi - lo > a.max_nodes || (s == 0 && lo != 0) ||
       (s == a.B - 1 && hi != a.T)) {
@@ -39,9 +39,10 @@ __global__ void __launch_bounds__(kThreads) snapshot_verify_kernel(VerifyArgs a,
   const size_t state = (size_t)dv * dk;
   for (int n = 0; n < hi - lo; ++n) {
     const size_t node = (size_t)(lo + n) * H + h;
+    const size_t qk_row = ((size_t)(lo + n) * a.Hk + kh) * dk;
     for (int j = t; j < dk; j += kThreads) {
-      qn[j] = to_f32(q[node * dk + j]);
-      kn[j] = to_f32(k[node * dk + j]);
+      qn[j] = to_f32(q[qk_row + j]);
+      kn[j] = to_f32(k[qk_row + j]);
     }
     for (int j = t; j < dv; j += kThreads) vn[j] = to_f32(v[node * dv + j]);
     if (t == 0) {
@@ -87,7 +88,7 @@ __global__ void __launch_bounds__(kThreads) snapshot_verify_kernel(VerifyArgs a,
         o = fmaf(x.w, qn[4 * j + 3], o);
       }
       static_cast<Tout *>(a.out)[node * dv + t] = from_f32<Tout>(o);
-      a.U[node * dv + t] = u;
+      store_u(a.U, node * dv + t, u, a.u_bf16);
     }
     __syncthreads();   // qn / kn / vn are rewritten for the next node
   }

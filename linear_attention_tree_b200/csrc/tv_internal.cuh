@@ -30,37 +30,53 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
   return __float2bfloat16_rn(x);
 }
 
-// Everything a verify kernel needs, by value.
+// Everything a verify kernel needs, by value.  Hk = number of q / k heads (value head h
+// reads q / k head h / (H / Hk)); u_bf16: U is stored as bf16.
 struct VerifyArgs {
   const void *q, *k, *v;
   const float *log_a, *b;
   const int32_t *parent, *node_offsets;
   const float *S_root;
   void *out;
-  float *U;
+  void *U;
   int *ws;
   int B, H, dk, dv, T, max_nodes;
+  int Hk, u_bf16;
 };
 
 struct CommitArgs {
-  const float *U;
+  const void *U;
   const void *k;
   const float *log_a, *S_root;
   const int32_t *node_offsets, *accepted_path, *parent;
   float *S_new;
   int *ws;
   int B, H, dk, dv, T, max_nodes, max_path;
+  int Hk, u_bf16;
 };
+
+// q / k head of value head h.
+__host__ __device__ __forceinline__ int qk_head(int h, int H, int Hk) { return h / (H / Hk); }
+
+// Element i of U in its storage type.
+__device__ __forceinline__ void store_u(void *U, size_t i, float x, int u_bf16) {
+  if (u_bf16) static_cast<__nv_bfloat16 *>(U)[i] = __float2bfloat16_rn(x);
+  else __stcs(static_cast<float *>(U) + i, x);
+}
+__device__ __forceinline__ float load_u(const void *U, size_t i, int u_bf16) {
+  return u_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16 *>(U)[i])
+                : static_cast<const float *>(U)[i];
+}
 
 // The commit that a fused commit + verify launch applies to S_root before verifying: the
 // previous step's tree, its pseudo-values and its accepted paths (one row per sequence).
 struct FuseArgs {
-  const float *U;                    // previous step's U
+  const void *U;                     // previous step's U (u_bf16: bf16)
   const void *k;                     // previous step's k (bf16)
   const float *log_a;
   const int32_t *node_offsets, *accepted_path, *parent;   // parent may be NULL
   float *S_new;                      // may be S_root
-  int T, max_nodes, max_path;
+  int T, max_nodes, max_path, u_bf16;
 };
 
 struct MetaArgs {

@@ -232,15 +232,15 @@ __device__ __forceinline__ void fuse_gather_path(Misc &ms, const FuseArgs &f, in
 
 // All threads: the u and k rows, log_a and the parent chain of the path entries.
 __device__ __forceinline__ void fuse_load_rows(unsigned char *sm, Misc &ms, const FuseArgs &f,
-                                               int h, int H, int tid) {
+                                               int h, int H, int kh, int Hk, int tid) {
   const int m = ms.f_m, lo = ms.f_lo;
   float *cu = reinterpret_cast<float *>(sm + kOffS);
   float *kk = cu + kFuseMax * 128;
   const __nv_bfloat16 *k = static_cast<const __nv_bfloat16 *>(f.k);
   for (int idx = tid; idx < m * 128; idx += kThreads) {
-    const size_t node = (size_t)(lo + ms.f_prow[idx >> 7]) * H + h;
-    cu[idx] = f.U[node * 128 + (idx & 127)];
-    kk[idx] = __bfloat162float(k[node * 128 + (idx & 127)]);
+    const int row = lo + ms.f_prow[idx >> 7];
+    cu[idx] = load_u(f.U, ((size_t)row * H + h) * 128 + (idx & 127), f.u_bf16);
+    kk[idx] = __bfloat162float(k[((size_t)row * Hk + kh) * 128 + (idx & 127)]);
   }
   if (tid < m) {
     const int p = ms.f_prow[tid];
@@ -339,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint8_t *paths = reinterpret_cast<uint8_t *>(sm + kOffPath);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H;
-  const int s = blockIdx.x / H, h = blockIdx.x % H;
+  const int s = blockIdx.x / H, h = blockIdx.x % H, kh = qk_head(h, H, a.Hk);
   // launched with programmatic stream serialisation: the kernel before this one on the
   // stream may still be finishing; wait for it (and its memory) before the first global
   // read, and let the kernel after this one get its CTAs resident early
@@ -370,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       // nothing to verify in this sequence: the commit alone
       if (warp == kThreads / 32 - 1) fuse_gather_path(ms, f, s, a.B, lane);
       __syncthreads();
-      fuse_load_rows(sm, ms, f, h, H, tid);
+      fuse_load_rows(sm, ms, f, h, H, kh, a.Hk, tid);
       __syncthreads();
       if (tid == 0) fuse_prefix(ms, a.ws, s);
       __syncthreads();
@@ -399,8 +399,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     ptx::mbar_arrive_expect_tx(bar_tma, 6 * kTile * 128);
     for (int half = 0; half < 2; ++half) {
       const uint32_t hb = sbase + kOffQK + half * kHalf;
-      ptx::tma_load_3d(hb, &tm_q, bar_tma, half * 64, h, lo);
-      ptx::tma_load_3d(hb + kTile * 128, &tm_k, bar_tma, half * 64, h, lo);
+      ptx::tma_load_3d(hb, &tm_q, bar_tma, half * 64, kh, lo);
+      ptx::tma_load_3d(hb + kTile * 128, &tm_k, bar_tma, half * 64, kh, lo);
       ptx::tma_load_3d(sbase + kOffV + half * kVHalf, &tm_v, bar_tma, half * 64, h, lo);
     }
   }
@@ -427,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const bool bad_tree = __syncthreads_or(bad) != 0;
   ptx::tc_fence_after();
   const uint32_t tmem = ms.tmem_base;
-  if (kFused) fuse_load_rows(sm, ms, f, h, H, tid);   // landed by the update before step 3's conversion
+  if (kFused) fuse_load_rows(sm, ms, f, h, H, kh, a.Hk, tid);   // landed by the update before step 3's conversion
 
   // ---- 2. Gram MMA once q / k have landed; tree walk ------------------------------------
   if (tid == kThreads - 1) {
@@ -575,8 +575,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int lo2 = a.node_offsets[s2];
       if (lo2 >= 0 && lo2 < a.T)
         for (int half = 0; half < 2; ++half) {
-          ptx::prefetch_tile_l2(&tm_q, half * 64, h2, lo2);
-          ptx::prefetch_tile_l2(&tm_k, half * 64, h2, lo2);
+          ptx::prefetch_tile_l2(&tm_q, half * 64, qk_head(h2, H, a.Hk), lo2);
+          ptx::prefetch_tile_l2(&tm_k, half * 64, qk_head(h2, H, a.Hk), lo2);
           ptx::prefetch_tile_l2(&tm_v, half * 64, h2, lo2);
         }
     }
@@ -705,20 +705,20 @@ __global__ void __launch_bounds__(kThreads, 2)
     ptx::tmem_wait_ld();
     release_tmem(warp, tmem);
     Tout *out = static_cast<Tout *>(a.out) + ((size_t)lo * H + h) * 128 + v;
-    float *U = a.U + ((size_t)lo * H + h) * 128 + v;
+    const size_t ub = ((size_t)lo * H + h) * 128 + v;
     const size_t rs = (size_t)H * 128;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       if (j0 + j < n_nodes) {
         st_out(out + (j0 + j) * rs, o0[j]);
-        __stcs(U + (j0 + j) * rs, u0[j]);
+        store_u(a.U, ub + (j0 + j) * rs, u0[j], a.u_bf16);
       }
     }
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       if (j0 + 16 + j < n_nodes) {
         st_out(out + (j0 + 16 + j) * rs, o1[j]);
-        __stcs(U + (j0 + 16 + j) * rs, u1[j]);
+        store_u(a.U, ub + (j0 + 16 + j) * rs, u1[j], a.u_bf16);
       }
     }
   }
@@ -731,7 +731,7 @@ cudaError_t launch_tc_t(const VerifyArgs &a, const FuseArgs &f, cudaStream_t st)
   // (a next tree with no nodes at all still gets maps over a one-row view: the kernel only
   // commits then)
   const int rows = a.T > 0 ? a.T : 1;
-  if (!make_node_map(&mq, a.q, a.H, rows, kTile) || !make_node_map(&mk, a.k, a.H, rows, kTile) ||
+  if (!make_node_map(&mq, a.q, a.Hk, rows, kTile) || !make_node_map(&mk, a.k, a.Hk, rows, kTile) ||
       !make_node_map(&mv, a.v, a.H, rows, kTile))
     return cudaErrorInvalidValue;
   auto kern = verify_tc_kernel<kGdn, Tout, kFused>;

@@ -144,14 +144,14 @@ __device__ __forceinline__ void row_coefficients(Meta &mt, int n, int r, int d) 
 // of the box are zero-filled or belong to the next sequence, and are never used.
 __device__ __forceinline__ void issue_tile(uint32_t sbase, Meta &mt, const CUtensorMap *tq,
                                            const CUtensorMap *tk, const CUtensorMap *tv_, int h,
-                                           int lo, int t) {
+                                           int kh, int lo, int t) {
   const int b = t & 1;
   const uint32_t bar = ptx::smem_addr(&mt.bar_t[b]);
   ptx::mbar_arrive_expect_tx(bar, 6 * kKHalf);
   for (int half = 0; half < 2; ++half) {
     const uint32_t hb = sbase + kOffQK + b * kQKBytes + half * kHalf;
-    ptx::tma_load_3d(hb, tq, bar, half * 64, h, lo + kTile * t);
-    ptx::tma_load_3d(hb + kKHalf, tk, bar, half * 64, h, lo + kTile * t);
+    ptx::tma_load_3d(hb, tq, bar, half * 64, kh, lo + kTile * t);
+    ptx::tma_load_3d(hb + kKHalf, tk, bar, half * 64, kh, lo + kTile * t);
     ptx::tma_load_3d(sbase + kOffV + b * kKBytes + half * kKHalf, tv_, bar, half * 64, h,
                      lo + kTile * t);
   }
@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   Meta &mt = *reinterpret_cast<Meta *>(sm + kOffMeta);
   const int tid = threadIdx.x, warp = tid >> 5;
   const int H = a.H;
-  const int s = blockIdx.x / H, h = blockIdx.x % H;
+  const int s = blockIdx.x / H, h = blockIdx.x % H, kh = qk_head(h, H, a.Hk);
   // launched with programmatic stream serialisation: wait for the previous kernel before
   // the first global access, and let the next one get its CTAs resident early
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_arrive_expect_tx(bs, 4 * kAtom2);
     for (int c = 0; c < 4; ++c)
       ptx::tma_load_2d(sbase + kOffS + c * kAtom2, &tm_s, bs, c * 32, blockIdx.x * 128);
-    for (int t = 0; t < 2 && t < n_tiles; ++t) issue_tile(sbase, mt, &tm_q, &tm_k, &tm_v, h, lo, t);
+    for (int t = 0; t < 2 && t < n_tiles; ++t) issue_tile(sbase, mt, &tm_q, &tm_k, &tm_v, h, kh, lo, t);
   }
   int t_issued = n_tiles < 2 ? n_tiles : 2;
   if (warp == 0) {
@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_arrive_expect_tx(bk, (n_tiles - 1) * kKBytes);
     for (int t = 0; t < n_tiles - 1; ++t)
       for (int half = 0; half < 2; ++half)
-        ptx::tma_load_3d(sbase + kOffKS + t * kKBytes + half * kKHalf, &tm_k, bk, half * 64, h,
+        ptx::tma_load_3d(sbase + kOffKS + t * kKBytes + half * kKHalf, &tm_k, bk, half * 64, kh,
                          lo + kTile * t);
   }
 
@@ -455,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     // q, k and v of this tile are consumed: the tile two ahead goes into this buffer
-    if (tid == 0 && c + 2 < n_tiles) issue_tile(sbase, mt, &tm_q, &tm_k, &tm_v, h, lo, c + 2);
+    if (tid == 0 && c + 2 < n_tiles) issue_tile(sbase, mt, &tm_q, &tm_k, &tm_v, h, kh, lo, c + 2);
     t_issued = c + 2 < n_tiles ? c + 3 : t_issued;
 
     // ---- 5. W rows (threads 0..63) and T rows (threads 128..191) of this tile ---------------
@@ -517,20 +517,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tmem_ld16(tlane + kColD + kTile + j0 + 16, u1);
       ptx::tmem_wait_ld();
       Tout *out = static_cast<Tout *>(a.out) + ((size_t)(lo + node0) * H + h) * 128 + v;
-      float *U = a.U + ((size_t)(lo + node0) * H + h) * 128 + v;
+      const size_t ub = ((size_t)(lo + node0) * H + h) * 128 + v;
       const size_t rs = (size_t)H * 128;
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         if (j0 + j < nc) {
           st_out(out + (j0 + j) * rs, o0[j]);
-          __stcs(U + (j0 + j) * rs, u0[j]);
+          store_u(a.U, ub + (j0 + j) * rs, u0[j], a.u_bf16);
         }
       }
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         if (j0 + 16 + j < nc) {
           st_out(out + (j0 + 16 + j) * rs, o1[j]);
-          __stcs(U + (j0 + 16 + j) * rs, u1[j]);
+          store_u(a.U, ub + (j0 + 16 + j) * rs, u1[j], a.u_bf16);
         }
       }
     }
@@ -546,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <bool kGdn, typename Tout>
 cudaError_t launch_tcw_t(const VerifyArgs &a, cudaStream_t st) {
   CUtensorMap mq, mk, mv, ms;
-  if (!make_node_map(&mq, a.q, a.H, a.T, kTile) || !make_node_map(&mk, a.k, a.H, a.T, kTile) ||
+  if (!make_node_map(&mq, a.q, a.Hk, a.T, kTile) || !make_node_map(&mk, a.k, a.Hk, a.T, kTile) ||
       !make_node_map(&mv, a.v, a.H, a.T, kTile) ||
       !make_state_map(&ms, a.S_root, (long long)a.B * a.H * 128))
     return cudaErrorInvalidValue;

@@ -129,10 +129,11 @@ def frontier_tree(seed: int, n: int, max_depth: int, fmax: int):
 class Workload:
     """One batch of draft trees with all per-node, per-head inputs (host numpy arrays).
 
-    Layouts (row-major, contiguous): q, k ``[T][H][dk]``; v ``[T][H][dv]``; log_a, b
-    ``[T][H]``; parent ``[T]`` (local index, -1 = root); node_offsets ``[B+1]``;
-    S_root ``[B][H][dv][dk]`` (row v, column k); accepted_path ``[B][max_path]``
-    (root-first local indices, -1 padded).
+    Layouts (row-major, contiguous): q, k ``[T][Hk][dk]`` (Hk = ``qk_heads``, H unless
+    several value heads share one q / k head: head h reads q / k head h // (H // Hk));
+    v ``[T][H][dv]``; log_a, b ``[T][H]``; parent ``[T]`` (local index, -1 = root);
+    node_offsets ``[B+1]``; S_root ``[B][H][dv][dk]`` (row v, column k);
+    accepted_path ``[B][max_path]`` (root-first local indices, -1 padded).
     """
     name: str
     mode: str                      # "gdn" or "scalar"
@@ -153,10 +154,15 @@ class Workload:
     accepted_path: np.ndarray
     max_nodes: int
     max_path: int
+    Hk: Optional[int] = None       # q / k heads; None = H
 
     @property
     def T(self) -> int:
         return int(self.node_offsets[-1])
+
+    @property
+    def qk_heads(self) -> int:
+        return self.H if self.Hk is None else self.Hk
 
     def seq_parent(self, s: int) -> np.ndarray:
         return self.parent[self.node_offsets[s]:self.node_offsets[s + 1]]
@@ -203,10 +209,11 @@ def synthetic(parents: List[List[int]], H: int, dk: int, dv: int, *, seed: int,
               mode: str = "gdn", in_dtype: str = "bf16", out_dtype: Optional[str] = None,
               paths: Optional[List[List[int]]] = None, log_a_mean: float = -4.0,
               s_std: float = 0.02, name: str = "synthetic",
-              max_nodes: Optional[int] = None) -> Workload:
+              max_nodes: Optional[int] = None, qk_heads: Optional[int] = None) -> Workload:
     """Workload for explicit per-sequence parent arrays with config-2 style distributions.
 
-    q, k ~ N(0,1) normalised per (node, head); v ~ N(0,1); b = sigmoid(N(0,1));
+    q, k ~ N(0,1) normalised per (node, q / k head), ``qk_heads`` of them (default H);
+    v ~ N(0,1); b = sigmoid(N(0,1));
     log_a = -softplus(N(log_a_mean, 0.5)); S_root ~ N(0, s_std).  In scalar mode the decay
     is one lambda per head (log_a = -softplus(N(log_a_mean, 0.5)) drawn per head) and b is
     absent.  ``paths`` defaults to the root->last-node path of every sequence.
@@ -217,9 +224,10 @@ def synthetic(parents: List[List[int]], H: int, dk: int, dv: int, *, seed: int,
     offsets = np.zeros(B + 1, dtype=np.int32)
     offsets[1:] = np.cumsum(counts)
     T = int(offsets[-1])
+    Hk = H if qk_heads is None else qk_heads
     S_root = (rng.standard_normal((B, H, dv, dk)) * s_std).astype(np.float32)
-    q = _unit_rows(rng.standard_normal((T, H, dk)).astype(np.float32))
-    k = _unit_rows(rng.standard_normal((T, H, dk)).astype(np.float32))
+    q = _unit_rows(rng.standard_normal((T, Hk, dk)).astype(np.float32))
+    k = _unit_rows(rng.standard_normal((T, Hk, dk)).astype(np.float32))
     v = rng.standard_normal((T, H, dv)).astype(np.float32)
     if mode == "gdn":
         b = _sigmoid(rng.standard_normal((T, H))).astype(np.float32)
@@ -238,7 +246,8 @@ def synthetic(parents: List[List[int]], H: int, dk: int, dv: int, *, seed: int,
     return Workload(name=name, mode=mode, B=B, H=H, dk=dk, dv=dv, in_dtype=in_dtype,
                     out_dtype=out_dtype or "f32", parent=parent, node_offsets=offsets,
                     q=q, k=k, v=v, log_a=log_a, b=b, S_root=S_root, accepted_path=ap,
-                    max_nodes=max([1] + counts), max_path=ap.shape[1])
+                    max_nodes=max([1] + counts), max_path=ap.shape[1],
+                    Hk=None if qk_heads is None else qk_heads)
 
 
 def _gdn_values(rng, T, H, dk, dv, B, log_a_mean):

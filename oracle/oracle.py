@@ -113,9 +113,13 @@ def walk(S_root: np.ndarray, path: Sequence[int], k, v, log_a, b, mode: str):
 
 
 def _head(w, s: int, h: int):
+    """Inputs of sequence s, value head h.  When several value heads share one q / k head
+    (``w.qk_heads`` < H, as in models whose value heads outnumber their key heads), head h
+    reads q / k head h // (H // qk_heads)."""
     lo, hi = int(w.node_offsets[s]), int(w.node_offsets[s + 1])
     f64 = lambda x: np.asarray(x, dtype=np.float64)
-    return (f64(w.q[lo:hi, h]), f64(w.k[lo:hi, h]), f64(w.v[lo:hi, h]),
+    kh = h // (w.H // getattr(w, "qk_heads", w.H))
+    return (f64(w.q[lo:hi, kh]), f64(w.k[lo:hi, kh]), f64(w.v[lo:hi, h]),
             f64(w.log_a[lo:hi, h]), None if w.b is None else f64(w.b[lo:hi, h]),
             f64(w.S_root[s, h]), w.parent[lo:hi])
 

@@ -37,8 +37,8 @@ def test_exports_every_declared_symbol():
 
 
 def test_problem_layout_and_version():
-    assert ctypes.sizeof(binding.Problem) == 44
-    assert L.lib().tv_version() >> 16 == 1
+    assert ctypes.sizeof(binding.Problem) == 52      # 13 int32 fields
+    assert L.lib().tv_version() >> 16 == 2
     assert binding.status_string(0) == "ok"
 
 
@@ -145,3 +145,15 @@ def test_commit_verify_checks_its_arguments():
     assert fn(ctypes.byref(prev), ptr(0), *[ptr(i) for i in range(1, 8)], ctypes.byref(other),
               *[ptr(i) for i in range(8, 15)], ptr(15), ptr(17), ptr(18), ctypes.c_size_t(256),
               None) == binding.TV_ERR_INVALID_ARG
+
+
+def test_grouped_heads_and_u_dtype_are_checked():
+    """qk_heads must divide H; bf16 U is refused by the CUDA-core kernel, which reads U back."""
+    import torch
+    for qk in (-1, 3, 5):
+        prob = L.make_problem(4, 4, 128, 128, 64, 16, 4, qk_heads=qk)
+        assert _call_verify(prob, _fake()) == binding.TV_ERR_INVALID_ARG, qk
+    prob = L.make_problem(4, 4, 64, 64, 64, 16, 4, u_dtype=torch.bfloat16)
+    assert _call_verify(prob, _fake()) == binding.TV_ERR_UNSUPPORTED
+    prob = L.make_problem(4, 4, 128, 128, 64, 16, 4, u_dtype=torch.bfloat16, kernel="simt")
+    assert _call_verify(prob, _fake()) == binding.TV_ERR_UNSUPPORTED

@@ -487,6 +487,25 @@ def test_meta_pin_catches_planted_mistakes(monkeypatch, mutant):
         pin_meta_varied_decay()
 
 
+def test_grouped_qk_heads_equal_repeated_qk():
+    """Value heads that share a q / k head give exactly what separate heads holding copies
+    of that q / k give (the ungrouped oracle, on an independently expanded workload)."""
+    rng = np.random.default_rng(51)
+    pars = [W.uniform_parent_tree(rng, 9, 4), W.uniform_parent_tree(rng, 6, 3)]
+    w = W.synthetic(pars, H=6, dk=8, dv=5, seed=51, qk_heads=2, in_dtype="f32")
+    assert w.q.shape == (w.T, 2, 8) and w.qk_heads == 2
+    e = W.synthetic(pars, H=6, dk=8, dv=5, seed=51, in_dtype="f32")
+    for name in ("v", "log_a", "b", "S_root", "parent", "node_offsets", "accepted_path"):
+        setattr(e, name, getattr(w, name))
+    e.q = np.repeat(w.q, 3, axis=1)     # value heads 0-2 share q / k head 0, 3-5 head 1
+    e.k = np.repeat(w.k, 3, axis=1)
+    o, U = O.tree_verify(w)
+    o_e, U_e = O.tree_verify(e)
+    np.testing.assert_array_equal(o, o_e)
+    np.testing.assert_array_equal(U, U_e)
+    np.testing.assert_array_equal(O.tree_commit(w), O.tree_commit(e))
+
+
 def test_commit_empty_path_is_root_and_matches_node_states():
     rng = np.random.default_rng(41)
     par = W.uniform_parent_tree(rng, 10, 4)
