@@ -511,6 +511,8 @@ def run_b200(args, workloads):
                                                           1e6 * c_avg, 1e6 * max_s / args.steps)
         if world == 1 and not args.other_configs_off:
             line["other_workloads"] = other_workloads(args, L, dev, peak)
+        if world == 1 and not args.no_budget:
+            line["batch_budget"] = batch_budget(line, 1e6 * c_avg)
         if world == 1 and not args.no_cpu_baseline:
             got = tuple(t.float().cpu().numpy().astype(np.float64) for t in outs[0])
             line["cpu_baseline"] = cpu_baseline_and_self_check(workloads[0], got)
@@ -587,24 +589,29 @@ def other_workloads(args, L, dev, peak) -> dict:
                  torch.empty((x.T, x.H, x.dv), dtype=torch.float32, device=dev)) for x in ws_]
         ws = L.new_workspace(L.make_problem(w.B, w.H, w.dk, w.dv, w.T, w.max_nodes, w.max_path), dev)
 
-        def one(i):
+        def one(i, kernel):
             d, (o, U), x = ds[i % N_SETS], outs[i % N_SETS], ws_[i % N_SETS]
             L.tree_verify(d["q"], d["k"], d["v"], d["log_a"], d["b"], d["parent"],
                           d["node_offsets"], d["S_root"], max_nodes=x.max_nodes, out=o, U=U,
-                          workspace=ws, kernel=args.kernel)
-        for i in range(10):
-            one(i)
+                          workspace=ws, kernel=kernel)
+
+        def timed(kernel, n):
+            for i in range(10 if n > 20 else 3):
+                one(i, kernel)
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(n)]
+            for i, (e0, e1) in enumerate(ev):
+                e0.record()
+                one(i, kernel)
+                e1.record()
+            torch.cuda.synchronize(dev)
+            if L.get_status(ws) != 0:
+                raise RuntimeError(f"device status after workload {idx}")
+            return statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev) / 1e3
         n = 60
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(n)]
-        for i, (e0, e1) in enumerate(ev):
-            e0.record()
-            one(i)
-            e1.record()
-        torch.cuda.synchronize(dev)
-        if L.get_status(ws) != 0:
-            raise RuntimeError(f"device status after workload {idx}")
-        t = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev) / 1e3
+        t = timed(args.kernel, n)
+        # the CUDA-core kernel on the same batches, for comparison
+        t_simt = timed("simt", 12) if args.kernel != "simt" else t
         vb = statistics.mean(verify_bytes(x) for x in ws_)
         T = statistics.mean(x.T for x in ws_)
         kname = ("verify_tc" if w.max_nodes <= 64 else "verify_tcw") if args.kernel != "simt" \
@@ -614,10 +621,55 @@ def other_workloads(args, L, dev, peak) -> dict:
             "verify_nodes_per_s": T / t, "algorithmic_bytes_per_launch": int(vb),
             "achieved_GBps": vb / t / 1e9, "frac_of_measured": vb / t / 1e9 / peak,
             "frac_of_8TBps": vb / t / 1e9 / NOMINAL_HBM_GBS,
-            "timing": f"CUDA events around each of {n} launches, {N_SETS} rotating input sets"}
+            "timing": f"CUDA events around each of {n} launches, {N_SETS} rotating input sets",
+            "verify_simt_us": 1e6 * t_simt, "speedup_vs_simt": t_simt / t}
         del ds, outs
         torch.cuda.empty_cache()
     return res
+
+
+def batch_budget(line: dict, commit_us: float) -> dict:
+    """The batch-wide verification budget on this GPU: fit the verify cost model, check its
+    predictions against this run's measured launches, and let it choose the budget for a
+    synthetic draft batch (128 trees of 64 nodes with acceptance estimates), the step being
+    this layer's verify plus its measured commit."""
+    import numpy as np
+    from linear_attention_tree_b200 import budget as Bd
+    from linear_attention_tree_b200 import workloads as W
+    model, samples = Bd.calibrate(launches=8)
+    fit_err = max(abs(model.predict_us(z, h) / us - 1) for z, h, us in samples)
+    checks = {}
+    measured = {"config3": line["verify_us"]}
+    for name, rec in line.get("other_workloads", {}).items():
+        measured[name] = rec["verify_us"]
+    for name, us in measured.items():
+        w = W.config(int(name[-1]), 0)
+        pred = model.predict_us([int(x) for x in np.diff(w.node_offsets)], w.H)
+        checks[name] = {"predicted_us": pred, "measured_us": us, "rel_err": pred / us - 1}
+    parents = [W.frontier_tree(900 + s, 64, 8, 4)[0] for s in range(128)]
+    trees = [(par, W.acceptance_estimates(par, 900 + s)) for s, par in enumerate(parents)]
+    pick = Bd.choose_budget(trees, 32, model, fixed_us=commit_us)
+    def rate(keeps):
+        sizes = [len(k) for k in keeps]
+        return Bd.expected_tokens(trees, keeps) / (commit_us + model.predict_us(sizes, 32))
+    all_nodes = [np.arange(64) for _ in trees]
+    raw = np.random.Generator(np.random.PCG64(4000)).integers(8, 49, size=128)
+    capped = [np.arange(int(n)) for n in Bd.cap_largest(np.minimum(raw, 64), 3072)]
+    greedy_3072 = Bd.select_nodes(trees, 3072, min_nodes=1)
+    return {
+        "model_us": {"tc": model.tc, "wide": model.wide,
+                     "features": "tc: 1, B*H, T*H; wide: 1, B*H, T*H, H*sum(ceil(n/64))"},
+        "fit_samples": len(samples), "fit_max_rel_err": fit_err,
+        "prediction_vs_this_run": checks,
+        "example": {
+            "batch": "128 frontier trees of 64 nodes, depth<=8, acceptance Beta(4,2)*0.6^rank",
+            "step": f"verify + this run's commit ({commit_us:.1f} us), one layer",
+            "chosen_budget_nodes": pick["budget"], "predicted_verify_us": pick["us"] - commit_us,
+            "expected_tokens": pick["tokens"], "tokens_per_us": pick["tokens_per_us"],
+            "verify_everything_tokens_per_us": rate(all_nodes),
+            "greedy_3072_tokens_per_us": rate(greedy_3072),
+            "index_prefix_cap_largest_3072_tokens_per_us": rate(capped)},
+    }
 
 
 CASES = {
@@ -682,6 +734,8 @@ def main(argv=None):
                     help="skip the per-node-snapshot baseline (4.3 GB of snapshots)")
     ap.add_argument("--other-configs-off", action="store_true",
                     help="skip the per-launch timing of the ragged and wide-tree workloads")
+    ap.add_argument("--no-budget", action="store_true",
+                    help="skip the cost-model calibration and the batch-budget example")
     ap.add_argument("--case", choices=sorted(CASES),
                     help="only launch one operation --launches times on one workload (for a "
                          "profiler): verifyN = tv_tree_verify on workload N, commit3, fused3 = "

@@ -35,7 +35,7 @@ import numpy as np
 
 __all__ = [
     "Workload", "config", "synthetic", "bf16_round", "bf16_bits", "frontier_tree",
-    "uniform_parent_tree", "depths_of", "CONFIG_NAMES",
+    "uniform_parent_tree", "depths_of", "acceptance_estimates", "CONFIG_NAMES",
 ]
 
 CONFIG_NAMES = {
@@ -125,6 +125,22 @@ def frontier_tree(seed: int, n: int, max_depth: int, fmax: int):
         attempt += 1
 
 
+def acceptance_estimates(parent: Sequence[int], seed: int) -> np.ndarray:
+    """Synthetic per-node acceptance estimates for a draft tree (float64 in (0, 1)).
+
+    Node n of sibling rank r (0 for its parent's first child, in index order) gets
+    Beta(4, 2) * 0.6**r: the first child is the drafter's top guess and its siblings are
+    successively less likely, as in a top-k expansion.
+    """
+    rng = _rng(seed)
+    seen: dict = {}
+    rank = np.empty(len(parent), dtype=np.int64)
+    for i, p in enumerate(parent):
+        rank[i] = seen.get(int(p), 0)
+        seen[int(p)] = rank[i] + 1
+    return rng.beta(4.0, 2.0, size=len(parent)) * 0.6 ** rank
+
+
 @dataclasses.dataclass
 class Workload:
     """One batch of draft trees with all per-node, per-head inputs (host numpy arrays).
@@ -166,6 +182,28 @@ class Workload:
 
     def seq_parent(self, s: int) -> np.ndarray:
         return self.parent[self.node_offsets[s]:self.node_offsets[s + 1]]
+
+    def subset(self, parent: np.ndarray, node_offsets: np.ndarray, rows: np.ndarray,
+               paths: Optional[List[List[int]]] = None) -> "Workload":
+        """The same sequences with only some nodes: ``rows`` are the kept nodes' rows in this
+        batch, ``parent`` / ``node_offsets`` the kept trees (local, topological).  The
+        per-node inputs are gathered row by row; S_root is shared.  ``paths`` (root-first,
+        local to the kept trees) default to the root->last-node path of every sequence."""
+        rows = np.asarray(rows, dtype=np.int64)
+        B = len(node_offsets) - 1
+        if B != self.B or int(node_offsets[-1]) != len(rows) or len(parent) != len(rows):
+            raise ValueError("subset does not describe this batch")
+        parents = [list(parent[node_offsets[s]:node_offsets[s + 1]]) for s in range(B)]
+        if paths is None:
+            paths = [(_path_to(p, len(p) - 1) if len(p) else []) for p in parents]
+        ap = _pad_paths(paths)
+        counts = np.diff(node_offsets)
+        return dataclasses.replace(
+            self, name=self.name + "-subset", parent=np.asarray(parent, dtype=np.int32),
+            node_offsets=np.asarray(node_offsets, dtype=np.int32), q=self.q[rows],
+            k=self.k[rows], v=self.v[rows], log_a=self.log_a[rows],
+            b=None if self.b is None else self.b[rows], accepted_path=ap,
+            max_nodes=max([1] + [int(c) for c in counts]), max_path=ap.shape[1])
 
     def depth_histogram(self) -> dict:
         hist: dict = {}
