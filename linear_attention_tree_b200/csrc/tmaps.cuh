@@ -49,4 +49,20 @@ inline bool make_state_map(CUtensorMap *m, const float *ptr, long long rows) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [T][H][128] output rows (fp32, or bf16 if `bf16`) as a 3-D tensor (128, H, T); box = a
+// whole 128-element row x 1 head x `rows` nodes, no swizzle: the box is `rows` node rows
+// laid out one after another in shared memory.
+inline bool make_row_map(CUtensorMap *m, void *ptr, bool bf16, int H, int T, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t es = bf16 ? 2 : 4;
+  cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)T};
+  cuuint64_t strides[2] = {128 * es, (cuuint64_t)H * 128 * es};
+  cuuint32_t box[3] = {128, 1, (cuuint32_t)rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr,
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace tv

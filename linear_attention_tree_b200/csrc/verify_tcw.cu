@@ -18,10 +18,13 @@
 //      then the k tiles of tiles 0..N/64-2 into the freed staging area, where the Gram
 //      blocks of later tiles read them.
 //   for every tile c:
-//   2. Gram blocks [Q_c ; K_c] . K_c'^T (tcgen05 kind::f16, 128 x 64 x 128), for each c' <= c
-//      that holds path nodes of tile c; the entries are stored by path position: q_n.k_i
-//      for i on path(n) (this tile's rows), b_n k_n.k_i for i in anc(n) (kept for all nodes).
-//   3. state MMA S_root . [Q_c ; K_c]^T (kind::f16, A = S_root from tensor memory).
+//   2. Gram blocks [Q_c ; K_c] . K_c'^T (tcgen05 kind::f16) for every c' <= c in one batch:
+//      the earlier tiles' k rows lie back to back in shared memory, so they form one operand
+//      of 64 c rows (one MMA chain, N = 64 c), and the tile's own k rows another (N = 64).
+//      The entries are stored by path position: q_n.k_i for i on path(n) (this tile's rows),
+//      b_n k_n.k_i for i in anc(n) (kept for all nodes).
+//   3. state MMA S_root . [Q_c ; K_c]^T (kind::f16, A = S_root from tensor memory), in the
+//      same batch as the Gram chains when their columns do not overlap its own.
 //   4. per value lane: o columns scaled by gamma_n, R^T_c[v][j] = b_j v_j[v] - b_j gamma_j
 //      (S_root k_j)[v] (tf32) into tensor memory next to the R^T of earlier tiles, U zeroed.
 //   5. T and W rows of the tile's nodes (register recursions, paths up to kDepth deep).
@@ -29,7 +32,10 @@
 //      (kind::tf32, A = R^T_c' from tensor memory, B = the coefficient block in shared memory).
 //   7. o_c and U_c from tensor memory to 128-byte row segments.
 // Tensor memory (512 columns): [0, 256) R^T of the four tiles, [256, 384) o^T | U^T of the
-// current tile, [384, 448) S_root in bf16, [448, 512) one Gram block.
+// current tile, [384, 448) S_root in bf16, [448, 512) the Gram block of the tile's own k rows.
+// The Gram blocks of tile c against tiles 0..c-1 go to [64 c, 128 c): R^T columns of tiles
+// c.. (written later, in step 4) and, for c = 3, the o^T | U^T columns (the state MMA then
+// waits until they are read).
 // Trees deeper than kDepth are verified by the CUDA-core algorithm in the same CTA.
 //
 // Every wait is bounded: a wait that runs out records TV_ERR_TIMEOUT on the status word; the
@@ -63,15 +69,16 @@ constexpr int kOffQK = 0;                   // two buffers (tile c in buffer c &
 constexpr int kOffV = 2 * kQKBytes;         // two buffers
 constexpr int kOffWT = kOffV + 2 * kKBytes; // [W ; T] block: 128 rows x 64 fp32, two K atoms
 constexpr int kOffKS = kOffWT + 2 * kAtom2; // k tiles 0..2 for the Gram blocks of later tiles
+constexpr int kKSHalf = 3 * kKHalf;         // K half h of those tiles: rows of tiles 0..2 in order
 constexpr int kOffS = kOffWT;               // S_root fp32 staging (64 KiB) before steps 2..7
 constexpr int kOffMeta = kOffKS + 3 * kKBytes;
 
 struct Meta {
-  unsigned long long bar_s, bar_t[2], bar_ks, bar_mma;
+  unsigned long long bar_s, bar_t[2], bar_ks, bar_mma, bar_g;
   uint32_t tmem_base;
   int flag;
   int maxdep;
-  int blk[kTiles];                    // tile c' holds path nodes of the current tile
+  unsigned blkm[kTiles];              // tile c: bit c' set if tile c' holds path nodes of its nodes
   unsigned long long anc[kNodes][4];  // strict-ancestor bits, word w = nodes 64 w .. 64 w + 63
   int par[kNodes];
   int dep[kNodes];
@@ -96,12 +103,12 @@ __device__ __forceinline__ int op2_off(int row, int k) {
 __device__ __forceinline__ float tf32_rn(float x) {
   return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
 }
+__device__ __forceinline__ void st_out(float *p, float x) { __stcs(p, x); }
+__device__ __forceinline__ void st_out(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&b);
 }
-__device__ __forceinline__ void st_out(float *p, float x) { __stcs(p, x); }
-__device__ __forceinline__ void st_out(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
 
 // Thread 0 waits on `bar`; every thread learns whether it completed (and leaves the
 // tcgen05 fence for the caller).  A time-out is recorded once.
@@ -167,6 +174,7 @@ __device__ void bail_out(Meta &mt, uint32_t tmem, bool tmem_held, int t_issued, 
     for (int t = t_issued > 2 ? t_issued - 2 : 0; t < t_issued; ++t)
       ptx::mbar_wait_bounded(ptx::smem_addr(&mt.bar_t[t & 1]), (t >> 1) & 1, kSpinLimit);
   }
+  if (threadIdx.x == 0) ptx::bulk_wait();   // output rows still being copied out
   ptx::tc_fence_before();
   __syncthreads();
   if (tmem_held && (threadIdx.x >> 5) == 0) {
@@ -180,7 +188,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     verify_tcw_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v,
-                      const __grid_constant__ CUtensorMap tm_s, VerifyArgs a) {
+                      const __grid_constant__ CUtensorMap tm_s,
+                      const __grid_constant__ CUtensorMap tm_o,
+                      const __grid_constant__ CUtensorMap tm_u, VerifyArgs a) {
   extern __shared__ unsigned char smem_dyn[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
@@ -204,20 +214,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_tiles = (n + kTile - 1) / kTile;
   const uint32_t sbase = ptx::smem_addr(sm);
 
-  // ---- 0. copies out, tensor memory, tree inputs and walk ---------------------------------
+  // ---- 0. tree inputs, copies out, tensor memory, walk -------------------------------------
+  // the tree's small loads go out first, ahead of the bulk copies in the memory queues
+  int p_in = -1;
+  float la_in = 0.f, bb_in = 0.f;
+  if (tid < n) {
+    p_in = a.parent[lo + tid];
+    la_in = a.log_a[(size_t)(lo + tid) * H + h];
+    bb_in = kGdn ? a.b[(size_t)(lo + tid) * H + h] : 0.f;
+  }
   if (tid == 0) {
     ptx::mbar_init(ptx::smem_addr(&mt.bar_s), 1);
     ptx::mbar_init(ptx::smem_addr(&mt.bar_t[0]), 1);
     ptx::mbar_init(ptx::smem_addr(&mt.bar_t[1]), 1);
     ptx::mbar_init(ptx::smem_addr(&mt.bar_ks), 1);
     ptx::mbar_init(ptx::smem_addr(&mt.bar_mma), 1);
+    ptx::mbar_init(ptx::smem_addr(&mt.bar_g), 3);
     ptx::fence_mbar_init();
     mt.flag = 0;
     mt.maxdep = 0;
+    for (int t = 0; t < kTiles; ++t) mt.blkm[t] = 0u;
     ptx::prefetch_tmap(&tm_q);
     ptx::prefetch_tmap(&tm_k);
     ptx::prefetch_tmap(&tm_v);
     ptx::prefetch_tmap(&tm_s);
+    ptx::prefetch_tmap(&tm_o);
+    ptx::prefetch_tmap(&tm_u);
     const uint32_t bs = ptx::smem_addr(&mt.bar_s);
     ptx::mbar_arrive_expect_tx(bs, 4 * kAtom2);
     for (int c = 0; c < 4; ++c)
@@ -229,20 +251,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tmem_alloc(ptx::smem_addr(&mt.tmem_base), kTmemCols);
     ptx::tmem_relinquish();
   }
-  bool bad = false;
-  {
-    int p = -1;
-    float la = 0.f, bb = 0.f;
-    if (tid < n) {
-      p = a.parent[lo + tid];
-      bad = p < -1 || p >= tid;
-      la = a.log_a[(size_t)(lo + tid) * H + h];
-      bb = kGdn ? a.b[(size_t)(lo + tid) * H + h] : 0.f;
-    }
-    mt.par[tid] = p;
-    mt.la[tid] = la;
-    mt.bb[tid] = bb;
-  }
+  const bool bad = tid < n && (p_in < -1 || p_in >= tid);
+  mt.par[tid] = p_in;
+  mt.la[tid] = la_in;
+  mt.bb[tid] = bb_in;
   ptx::tc_fence_before();
   const bool bad_tree = __syncthreads_or(bad) != 0;
   ptx::tc_fence_after();
@@ -280,6 +292,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     mt.bg[tid] = mt.bb[tid] * gam;
     mt.bq[tid] = mt.bb[tid];
     atomicMax(&mt.maxdep, d);
+    // tiles holding path nodes (ancestors and the node itself), OR-ed over each warp: the
+    // 32 nodes of a warp lie in one tile
+    unsigned tm = tid < n ? 1u << (tid >> 6) : 0u;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) tm |= bits[w] ? 1u << w : 0u;
+    tm = __reduce_or_sync(0xffffffffu, tm);
+    if ((tid & 31) == 0 && tm) atomicOr(&mt.blkm[tid >> 6], tm);
   }
   __syncthreads();
   if (mt.maxdep > kDepth) {
@@ -322,11 +341,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_arrive_expect_tx(bk, (n_tiles - 1) * kKBytes);
     for (int t = 0; t < n_tiles - 1; ++t)
       for (int half = 0; half < 2; ++half)
-        ptx::tma_load_3d(sbase + kOffKS + t * kKBytes + half * kKHalf, &tm_k, bk, half * 64, kh,
+        ptx::tma_load_3d(sbase + kOffKS + half * kKSHalf + t * kKHalf, &tm_k, bk, half * 64, kh,
                          lo + kTile * t);
   }
 
-  uint32_t mma_phase = 0;
+  uint32_t mma_phase = 0, gphase = 0;
   for (int c = 0; c < n_tiles; ++c) {
     const int b = c & 1, node0 = c * kTile;
     const int nc = n - node0 < kTile ? n - node0 : kTile;
@@ -337,47 +356,64 @@ __global__ void __launch_bounds__(kThreads, 1)
       bail_out(mt, tmem, true, t_issued, ks_issued, false);
       return;
     }
-    // which tiles hold path nodes of this tile's nodes (word c' of anc | self)
-    if (tid < kTiles) mt.blk[tid] = 0;
-    __syncthreads();
-    if (tid < nc) {
-      const int nn = node0 + tid;
-      for (int c2 = 0; c2 <= c; ++c2) {
-        const unsigned long long wbits = mt.anc[nn][c2] | (c2 == c ? 1ull << tid : 0ull);
-        if (wbits) atomicOr(&mt.blk[c2], 1);
-      }
-    }
-    __syncthreads();
+    const unsigned blkm = mt.blkm[c];       // tiles holding path nodes of this tile's nodes
 
-    // ---- 2. Gram blocks and their entries by path position ---------------------------------
+    // ---- 2. Gram blocks and their entries by path position (+ 3. the state MMA) ----------
     const bool g_is_q = row < kTile;
     const int gr = row & (kTile - 1);
     const int gn = node0 + gr;               // node of this Gram row
     const bool g_live = gr < nc;
-    for (int c2 = 0; c2 <= c; ++c2) {
-      if (!mt.blk[c2]) continue;
-      if (tid == 0) {
-        ptx::tc_fence_after();
-        const bool own = c2 == c;
-        const uint32_t kb = own ? qk + kKHalf : sbase + kOffKS + c2 * kKBytes;
-        const uint32_t kstride = own ? kHalf : kKHalf;
+    const uint32_t col_early = kTile * c;    // Gram blocks against tiles 0..c-1
+    const bool state_early = 2 * kTile * c <= (int)kColD;
+    // Three chains into separate columns, issued by one thread each of warps 0-2 (the issue
+    // of a tcgen05.mma takes tens of cycles); every issuer commits to bar_g.
+    if ((tid & 31) == 0 && warp < 3) {
+      ptx::tc_fence_after();
+      if (warp == 0) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           ptx::mma_bf16(tmem + kColG,
                         ptx::smem_desc_sw128(qk + (kk >> 2) * kHalf + (kk & 3) * 32, 1024),
-                        ptx::smem_desc_sw128(kb + (kk >> 2) * kstride + (kk & 3) * 32, 1024),
-                        ptx::idesc_bf16_f32(128, 64), kk > 0 ? 1u : 0u);
-        ptx::mma_commit(ptx::smem_addr(&mt.bar_mma));
+                        ptx::smem_desc_sw128(qk + kKHalf + (kk >> 2) * kHalf + (kk & 3) * 32, 1024),
+                        ptx::idesc_bf16_f32(128, kTile), kk > 0 ? 1u : 0u);
+      } else if (warp == 1 && c > 0) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          ptx::mma_bf16(tmem + col_early,
+                        ptx::smem_desc_sw128(qk + (kk >> 2) * kHalf + (kk & 3) * 32, 1024),
+                        ptx::smem_desc_sw128(sbase + kOffKS + (kk >> 2) * kKSHalf + (kk & 3) * 32, 1024),
+                        ptx::idesc_bf16_f32(128, kTile * c), kk > 0 ? 1u : 0u);
+      } else if (warp == 2 && state_early) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          ptx::mma_bf16_tmem_a(tmem + kColD, tmem + kColA + kk * 8,
+                               ptx::smem_desc_sw128(qk + (kk >> 2) * kHalf + (kk & 3) * 32, 1024),
+                               ptx::idesc_bf16_f32(128, 128), kk > 0 ? 1u : 0u);
       }
-      if (!wait_all(mt, ptx::smem_addr(&mt.bar_mma), mma_phase++ & 1, a.ws, s)) {
-        bail_out(mt, tmem, true, t_issued, ks_issued, false);
-        return;
-      }
-      ptx::tc_fence_after();
+      ptx::mma_commit(ptx::smem_addr(&mt.bar_g));
+    }
+    // The previous tile's output rows must have been read out of shared memory before the
+    // extraction below writes its slots; then that tile's buffer takes the tile two ahead.
+    if (tid == 0) ptx::bulk_wait_read();
+    if (!wait_all(mt, ptx::smem_addr(&mt.bar_g), gphase++ & 1, a.ws, s)) {
+      bail_out(mt, tmem, true, t_issued, ks_issued, false);
+      return;
+    }
+    if (c >= 1 && c + 1 < n_tiles) {
+      if (tid == 0) issue_tile(sbase, mt, &tm_q, &tm_k, &tm_v, h, kh, lo, c + 1);
+      t_issued = c + 2;
+    }
+    ptx::tc_fence_after();
+    // Each thread stages its 32 Gram values of a block in its own 128-byte slot of the
+    // (idle) coefficient buffer, then visits only the columns on its row's path.
+    unsigned char *slot = sm + kOffWT + (row * 2 + ch) * 128;
+    for (int c2 = 0; c2 <= c; ++c2) {
+      if (!((blkm >> c2) & 1u)) continue;
       if (g_is_q || kGdn) {   // uniform per warp: rows 0..63 are q rows
+        const uint32_t gcol = c2 < c ? col_early + kTile * c2 : kColG;
         float g[2][16];
-        ptx::tmem_ld16(tlane + kColG + 32 * ch, g[0]);
-        ptx::tmem_ld16(tlane + kColG + 32 * ch + 16, g[1]);
+        ptx::tmem_ld16(tlane + gcol + 32 * ch, g[0]);
+        ptx::tmem_ld16(tlane + gcol + 32 * ch + 16, g[1]);
         ptx::tmem_wait_ld();
         if (g_live) {
           // bits of path(gn) (q rows) or anc(gn) (k rows) in tile c2, and the number of path
@@ -387,34 +423,45 @@ __global__ void __launch_bounds__(kThreads, 1)
           unsigned long long wb = mt.anc[gn][c2];
           if (g_is_q && c2 == c) wb |= 1ull << gr;
           pos += __popcll(wb & ((1ull << (32 * ch)) - 1ull));
-          const unsigned bits = (unsigned)(wb >> (32 * ch));
-          const float scale = g_is_q ? 1.f : mt.bb[gn];
+          unsigned bits = (unsigned)(wb >> (32 * ch));
+          if (bits) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if ((bits >> j) & 1u) {
-              if (g_is_q) mt.gpos[pos][gr] = g[j >> 4][j & 15];
-              else mt.lpos[pos][gn] = scale * g[j >> 4][j & 15];
+            for (int q4 = 0; q4 < 8; ++q4)
+              *reinterpret_cast<float4 *>(slot + ((q4 ^ (row & 7)) << 4)) =
+                  make_float4(g[q4 >> 2][(q4 & 3) * 4], g[q4 >> 2][(q4 & 3) * 4 + 1],
+                              g[q4 >> 2][(q4 & 3) * 4 + 2], g[q4 >> 2][(q4 & 3) * 4 + 3]);
+            const float scale = g_is_q ? 1.f : mt.bb[gn];
+            while (bits) {
+              const int j = __ffs(bits) - 1;
+              bits &= bits - 1u;
+              const float val =
+                  *reinterpret_cast<const float *>(slot + ((((j >> 2) ^ (row & 7)) << 4) | ((j & 3) << 2)));
+              if (g_is_q) mt.gpos[pos][gr] = val;
+              else mt.lpos[pos][gn] = scale * val;
               ++pos;
             }
+          }
         }
       }
-      ptx::tc_fence_before();
-      __syncthreads();
     }
+    ptx::tc_fence_before();
+    __syncthreads();
 
-    // ---- 3. state MMA: [o^T | U^T] columns = S_root . [Q_c ; K_c]^T -----------------------
-    if (tid == 0) {
-      ptx::tc_fence_after();
+    if (!state_early) {
+      // ---- 3. state MMA: [o^T | U^T] columns = S_root . [Q_c ; K_c]^T ---------------------
+      if (tid == 0) {
+        ptx::tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        ptx::mma_bf16_tmem_a(tmem + kColD, tmem + kColA + kk * 8,
-                             ptx::smem_desc_sw128(qk + (kk >> 2) * kHalf + (kk & 3) * 32, 1024),
-                             ptx::idesc_bf16_f32(128, 128), kk > 0 ? 1u : 0u);
-      ptx::mma_commit(ptx::smem_addr(&mt.bar_mma));
-    }
-    if (!wait_all(mt, ptx::smem_addr(&mt.bar_mma), mma_phase++ & 1, a.ws, s)) {
-      bail_out(mt, tmem, true, t_issued, ks_issued, false);
-      return;
+        for (int kk = 0; kk < 8; ++kk)
+          ptx::mma_bf16_tmem_a(tmem + kColD, tmem + kColA + kk * 8,
+                               ptx::smem_desc_sw128(qk + (kk >> 2) * kHalf + (kk & 3) * 32, 1024),
+                               ptx::idesc_bf16_f32(128, 128), kk > 0 ? 1u : 0u);
+        ptx::mma_commit(ptx::smem_addr(&mt.bar_mma));
+      }
+      if (!wait_all(mt, ptx::smem_addr(&mt.bar_mma), mma_phase++ & 1, a.ws, s)) {
+        bail_out(mt, tmem, true, t_issued, ks_issued, false);
+        return;
+      }
     }
     ptx::tc_fence_after();
 
@@ -454,10 +501,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    // q, k and v of this tile are consumed: the tile two ahead goes into this buffer
-    if (tid == 0 && c + 2 < n_tiles) issue_tile(sbase, mt, &tm_q, &tm_k, &tm_v, h, kh, lo, c + 2);
-    t_issued = c + 2 < n_tiles ? c + 3 : t_issued;
-
     // ---- 5. W rows (threads 0..63) and T rows (threads 128..191) of this tile ---------------
     if ((tid & 127) < kTile && (tid & 127) < nc) {
       const int r = tid & 63, nn = node0 + r, d = mt.dep[nn];
@@ -468,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- 6. path MMAs, one coefficient block per tile c' holding path nodes -----------------
     for (int c2 = 0; c2 <= c; ++c2) {
-      if (!mt.blk[c2]) continue;
+      if (!((blkm >> c2) & 1u)) continue;
       {
         // thread t writes K atom t / 128 (node columns 32 atom .. 32 atom + 31 of tile c2) of
         // operand row t % 128: zeros, then its path coefficients that fall there
@@ -516,27 +559,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tmem_ld16(tlane + kColD + kTile + j0, u0);
       ptx::tmem_ld16(tlane + kColD + kTile + j0 + 16, u1);
       ptx::tmem_wait_ld();
-      Tout *out = static_cast<Tout *>(a.out) + ((size_t)(lo + node0) * H + h) * 128 + v;
-      const size_t ub = ((size_t)(lo + node0) * H + h) * 128 + v;
-      const size_t rs = (size_t)H * 128;
+      if (nc == kTile) {
+        // a full tile: node rows into shared memory (o over the coefficient buffer, U over
+        // this tile's dead q / k buffer), then one tensor store each; both buffers are read
+        // out before the next tile touches them
+        Tout *ost = reinterpret_cast<Tout *>(sm + kOffWT);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        if (j0 + j < nc) {
-          st_out(out + (j0 + j) * rs, o0[j]);
-          store_u(a.U, ub + (j0 + j) * rs, u0[j], a.u_bf16);
+        for (int j = 0; j < 16; ++j) {
+          ost[(j0 + j) * 128 + v] = from_f32<Tout>(o0[j]);
+          ost[(j0 + 16 + j) * 128 + v] = from_f32<Tout>(o1[j]);
         }
-      }
+        unsigned char *ust = sm + kOffQK + b * kQKBytes;
+        if (a.u_bf16) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        if (j0 + 16 + j < nc) {
-          st_out(out + (j0 + 16 + j) * rs, o1[j]);
-          store_u(a.U, ub + (j0 + 16 + j) * rs, u1[j], a.u_bf16);
+          for (int j = 0; j < 16; ++j) {
+            reinterpret_cast<__nv_bfloat16 *>(ust)[(j0 + j) * 128 + v] = __float2bfloat16_rn(u0[j]);
+            reinterpret_cast<__nv_bfloat16 *>(ust)[(j0 + 16 + j) * 128 + v] = __float2bfloat16_rn(u1[j]);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            reinterpret_cast<float *>(ust)[(j0 + j) * 128 + v] = u0[j];
+            reinterpret_cast<float *>(ust)[(j0 + 16 + j) * 128 + v] = u1[j];
+          }
+        }
+        ptx::fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+          ptx::tma_store_3d(&tm_o, sbase + kOffWT, 0, h, lo + node0);
+          ptx::tma_store_3d(&tm_u, ptx::smem_addr(ust), 0, h, lo + node0);
+          ptx::bulk_commit();
+        }
+      } else {
+        Tout *out = static_cast<Tout *>(a.out) + ((size_t)(lo + node0) * H + h) * 128 + v;
+        const size_t ub = ((size_t)(lo + node0) * H + h) * 128 + v;
+        const size_t rs = (size_t)H * 128;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          if (j0 + j < nc) {
+            st_out(out + (j0 + j) * rs, o0[j]);
+            store_u(a.U, ub + (j0 + j) * rs, u0[j], a.u_bf16);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          if (j0 + 16 + j < nc) {
+            st_out(out + (j0 + 16 + j) * rs, o1[j]);
+            store_u(a.U, ub + (j0 + 16 + j) * rs, u1[j], a.u_bf16);
+          }
         }
       }
     }
     ptx::tc_fence_before();
     __syncthreads();
   }
+  if (tid == 0) ptx::bulk_wait();
   if (warp == 0) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
@@ -545,10 +622,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <bool kGdn, typename Tout>
 cudaError_t launch_tcw_t(const VerifyArgs &a, cudaStream_t st) {
-  CUtensorMap mq, mk, mv, ms;
+  CUtensorMap mq, mk, mv, ms, mo, mu;
   if (!make_node_map(&mq, a.q, a.Hk, a.T, kTile) || !make_node_map(&mk, a.k, a.Hk, a.T, kTile) ||
       !make_node_map(&mv, a.v, a.H, a.T, kTile) ||
-      !make_state_map(&ms, a.S_root, (long long)a.B * a.H * 128))
+      !make_state_map(&ms, a.S_root, (long long)a.B * a.H * 128) ||
+      !make_row_map(&mo, a.out, sizeof(Tout) == 2, a.H, a.T, kTile) ||
+      !make_row_map(&mu, a.U, a.u_bf16 != 0, a.H, a.T, kTile))
     return cudaErrorInvalidValue;
   auto kern = verify_tcw_kernel<kGdn, Tout>;
   cudaError_t e =
@@ -564,7 +643,7 @@ cudaError_t launch_tcw_t(const VerifyArgs &a, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, ms, a);
+  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, ms, mo, mu, a);
 }
 
 }  // namespace
