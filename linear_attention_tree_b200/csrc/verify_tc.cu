@@ -330,7 +330,9 @@ template <bool kGdn, typename Tout, bool kFused>
 __global__ void __launch_bounds__(kThreads, 2)
     verify_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, VerifyArgs a, FuseArgs f,
+                     const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_o,
+                     const __grid_constant__ CUtensorMap tm_u, VerifyArgs a, FuseArgs f,
                      int prefetch_stride) {
   extern __shared__ unsigned char smem_dyn[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
@@ -389,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     ptx::mbar_init(bar_tma, 1);
     ptx::mbar_init(bar_gram, 1);
     ptx::mbar_init(bar_state, 1);
-    ptx::mbar_init(bar_sum, 1);
+    ptx::mbar_init(bar_sum, 2);
     ptx::fence_mbar_init();
     ms.flag = 0;
     ms.maxdep = 0;
@@ -678,13 +680,16 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
 
   // ---- 7. path-sum MMA: columns 0..127 += R^T . [W ; T]^T (tf32), i.e. o^T and U^T ------
-  if (tid == kThreads - 1) {
+  // two chains of N = 64 issued by two threads: W rows into the o columns, T rows into the
+  // U columns (rows 64.. of each K atom start 8 KiB into it)
+  if (tid == kThreads - 1 || tid == kThreads - 33) {
     ptx::tc_fence_after();
-    constexpr uint32_t idesc = ptx::idesc_tf32_f32(128, 128);
+    const uint32_t half = tid == kThreads - 1 ? 0u : 1u;
+    constexpr uint32_t idesc = ptx::idesc_tf32_f32(128, 64);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
-      ptx::mma_tf32_tmem_a(tmem, tmem + kColR + kk * 8,
-                           ptx::smem_desc_sw128(sbase + kOffA2 + (kk >> 2) * kAtom2 + (kk & 3) * 32, 1024),
+      ptx::mma_tf32_tmem_a(tmem + half * kTile, tmem + kColR + kk * 8,
+                           ptx::smem_desc_sw128(sbase + kOffA2 + half * (kTile * 128) + (kk >> 2) * kAtom2 + (kk & 3) * 32, 1024),
                            idesc, 1u);
     ptx::mma_commit(bar_sum);
   }
@@ -704,21 +709,56 @@ __global__ void __launch_bounds__(kThreads, 2)
     ptx::tmem_ld16(tlane + kTile + j0 + 16, u1);
     ptx::tmem_wait_ld();
     release_tmem(warp, tmem);
-    Tout *out = static_cast<Tout *>(a.out) + ((size_t)lo * H + h) * 128 + v;
-    const size_t ub = ((size_t)lo * H + h) * 128 + v;
-    const size_t rs = (size_t)H * 128;
+    if (n_nodes == kTile) {
+      // a full tree: node rows into shared memory (o over the dead [W ; T] operand, U over
+      // the dead S_root operand), then one tensor store each; the CTA leaves once they have
+      // been read out of shared memory
+      Tout *ost = reinterpret_cast<Tout *>(sm + kOffA2);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      if (j0 + j < n_nodes) {
-        st_out(out + (j0 + j) * rs, o0[j]);
-        store_u(a.U, ub + (j0 + j) * rs, u0[j], a.u_bf16);
+      for (int j = 0; j < 16; ++j) {
+        ost[(j0 + j) * 128 + v] = from_f32<Tout>(o0[j]);
+        ost[(j0 + 16 + j) * 128 + v] = from_f32<Tout>(o1[j]);
       }
-    }
+      if (a.u_bf16) {
+        __nv_bfloat16 *ust = reinterpret_cast<__nv_bfloat16 *>(sm + kOffS);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      if (j0 + 16 + j < n_nodes) {
-        st_out(out + (j0 + 16 + j) * rs, o1[j]);
-        store_u(a.U, ub + (j0 + 16 + j) * rs, u1[j], a.u_bf16);
+        for (int j = 0; j < 16; ++j) {
+          ust[(j0 + j) * 128 + v] = __float2bfloat16_rn(u0[j]);
+          ust[(j0 + 16 + j) * 128 + v] = __float2bfloat16_rn(u1[j]);
+        }
+      } else {
+        float *ust = reinterpret_cast<float *>(sm + kOffS);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          ust[(j0 + j) * 128 + v] = u0[j];
+          ust[(j0 + 16 + j) * 128 + v] = u1[j];
+        }
+      }
+      ptx::fence_proxy_async_smem();
+      __syncthreads();
+      if (tid == 0) {
+        ptx::tma_store_3d(&tm_o, sbase + kOffA2, 0, h, lo);
+        ptx::tma_store_3d(&tm_u, sbase + kOffS, 0, h, lo);
+        ptx::bulk_commit();
+        ptx::bulk_wait_read();
+      }
+    } else {
+      Tout *out = static_cast<Tout *>(a.out) + ((size_t)lo * H + h) * 128 + v;
+      const size_t ub = ((size_t)lo * H + h) * 128 + v;
+      const size_t rs = (size_t)H * 128;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (j0 + j < n_nodes) {
+          st_out(out + (j0 + j) * rs, o0[j]);
+          store_u(a.U, ub + (j0 + j) * rs, u0[j], a.u_bf16);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (j0 + 16 + j < n_nodes) {
+          st_out(out + (j0 + 16 + j) * rs, o1[j]);
+          store_u(a.U, ub + (j0 + 16 + j) * rs, u1[j], a.u_bf16);
+        }
       }
     }
   }
@@ -727,12 +767,14 @@ __global__ void __launch_bounds__(kThreads, 2)
 // ---- host side ------------------------------------------------------------------------
 template <bool kGdn, typename Tout, bool kFused>
 cudaError_t launch_tc_t(const VerifyArgs &a, const FuseArgs &f, cudaStream_t st) {
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo, mu;
   // (a next tree with no nodes at all still gets maps over a one-row view: the kernel only
   // commits then)
   const int rows = a.T > 0 ? a.T : 1;
   if (!make_node_map(&mq, a.q, a.Hk, rows, kTile) || !make_node_map(&mk, a.k, a.Hk, rows, kTile) ||
-      !make_node_map(&mv, a.v, a.H, rows, kTile))
+      !make_node_map(&mv, a.v, a.H, rows, kTile) ||
+      !make_row_map(&mo, a.out, sizeof(Tout) == 2, a.H, rows, kTile) ||
+      !make_row_map(&mu, a.U, a.u_bf16 != 0, a.H, rows, kTile))
     return cudaErrorInvalidValue;
   auto kern = verify_tc_kernel<kGdn, Tout, kFused>;
   cudaError_t e =
@@ -752,7 +794,7 @@ cudaError_t launch_tc_t(const VerifyArgs &a, const FuseArgs &f, cudaStream_t st)
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, a, f, 2 * sms);
+  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, mu, a, f, 2 * sms);
 }
 
 }  // namespace
