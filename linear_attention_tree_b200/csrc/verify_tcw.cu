@@ -74,7 +74,7 @@ constexpr int kOffS = kOffWT;               // S_root fp32 staging (64 KiB) befo
 constexpr int kOffMeta = kOffKS + 3 * kKBytes;
 
 struct Meta {
-  unsigned long long bar_s, bar_t[2], bar_ks, bar_mma, bar_g;
+  unsigned long long bar_s, bar_t[2], bar_ks, bar_mma, bar_g, bar_pm;
   uint32_t tmem_base;
   int flag;
   int maxdep;
@@ -230,6 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(ptx::smem_addr(&mt.bar_ks), 1);
     ptx::mbar_init(ptx::smem_addr(&mt.bar_mma), 1);
     ptx::mbar_init(ptx::smem_addr(&mt.bar_g), 3);
+    ptx::mbar_init(ptx::smem_addr(&mt.bar_pm), 2);
     ptx::fence_mbar_init();
     mt.flag = 0;
     mt.maxdep = 0;
@@ -345,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                          lo + kTile * t);
   }
 
-  uint32_t mma_phase = 0, gphase = 0;
+  uint32_t mma_phase = 0, gphase = 0, pm_phase = 0;
   for (int c = 0; c < n_tiles; ++c) {
     const int b = c & 1, node0 = c * kTile;
     const int nc = n - node0 < kTile ? n - node0 : kTile;
@@ -522,11 +523,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<float4 *>(sm + kOffWT + op2_off(r2, atom * 32 + q4 * 4)) = zf;
         const int r = r2 & 63;
         if (r < nc) {
-          const int nn = node0 + r, d = mt.dep[nn];
+          // the path positions that fall in tile c2: after the ones in tiles 0..c2-1
+          const int nn = node0 + r;
           const float(*cf)[kTile] = r2 < kTile ? mt.gpos : mt.tpos;
-          for (int a2 = 0; a2 < d; ++a2) {
+          int a0 = 0;
+          for (int w = 0; w < c2; ++w) a0 += __popcll(mt.anc[nn][w]);
+          const int a1 = a0 + __popcll(mt.anc[nn][c2]) + (c2 == c ? 1 : 0);
+          for (int a2 = a0; a2 < a1; ++a2) {
             const int i = mt.paths[a2][nn];
-            if ((i >> 6) == c2 && ((i >> 5) & 1) == atom)
+            if (((i >> 5) & 1) == atom)
               *reinterpret_cast<float *>(sm + kOffWT + op2_off(r2, i & 63)) = cf[a2][r];
           }
         }
@@ -534,16 +539,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncthreads();
-      if (tid == 0) {
+      // two chains of N = 64 from two threads: W rows into the o columns, T rows into the U
+      // columns (rows 64.. of each K atom start 8 KiB into it)
+      if (tid == 0 || tid == 32) {
         ptx::tc_fence_after();
+        const uint32_t hf = tid == 0 ? 0u : 1u;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          ptx::mma_tf32_tmem_a(tmem + kColD, tmem + kColR + kTile * c2 + kk * 8,
-                               ptx::smem_desc_sw128(sbase + kOffWT + (kk >> 2) * kAtom2 + (kk & 3) * 32, 1024),
-                               ptx::idesc_tf32_f32(128, 128), 1u);
-        ptx::mma_commit(ptx::smem_addr(&mt.bar_mma));
+          ptx::mma_tf32_tmem_a(tmem + kColD + hf * kTile, tmem + kColR + kTile * c2 + kk * 8,
+                               ptx::smem_desc_sw128(sbase + kOffWT + hf * (kTile * 128) + (kk >> 2) * kAtom2 + (kk & 3) * 32, 1024),
+                               ptx::idesc_tf32_f32(128, kTile), 1u);
+        ptx::mma_commit(ptx::smem_addr(&mt.bar_pm));
       }
-      if (!wait_all(mt, ptx::smem_addr(&mt.bar_mma), mma_phase++ & 1, a.ws, s)) {
+      if (!wait_all(mt, ptx::smem_addr(&mt.bar_pm), pm_phase++ & 1, a.ws, s)) {
         bail_out(mt, tmem, true, t_issued, ks_issued, false);
         return;
       }
