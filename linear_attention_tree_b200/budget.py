@@ -264,9 +264,9 @@ class CostModel:
 
 
 # Fitted on a B200 (SM clock 1965 MHz) by `calibrate()` with H = 32, dk = dv = 128, bf16
-# inputs, fp32 o and U, cold L2 before every launch: 13 batches, largest relative error of
-# the fit 5.7%; the bench workloads it did not see were predicted within 18%.
-B200_DEFAULT = CostModel(tc=(10.74, 0.03231, 0.000150), wide=(36.67, 0.0, 0.00170, 0.01264))
+# inputs, fp32 o and U, cold L2 before every launch: 14 batches, largest relative error of
+# the fit 7%; the three bench workloads, which it did not see, were predicted within 8%.
+B200_DEFAULT = CostModel(tc=(9.584, 0.03315, 0.0001474), wide=(32.77, 0.002634, 0.001159, 0.008996))
 
 
 def _prefix_curve(trees, H: int, model: CostModel, cap: Optional[int], min_nodes: int,
@@ -362,35 +362,38 @@ def measure_us(w, *, launches: int = 12, flush=None, kernel: str = "auto") -> fl
     return 1e3 * float(np.median([a.elapsed_time(b) for a, b in times]))
 
 
+# (B, smallest tree, largest tree, deepest path, most children of a node)
 CALIBRATION_BATCHES = (
-    (16, 8, 32), (32, 1, 8), (32, 33, 64), (64, 8, 48), (128, 8, 48), (128, 48, 64),
-    (256, 4, 24), (8, 64, 64), (2, 65, 128), (4, 128, 256), (8, 200, 256), (16, 65, 256),
-    (8, 8, 130),
+    (16, 8, 32, 8, 4), (32, 1, 8, 8, 4), (32, 33, 64, 8, 2), (64, 8, 48, 7, 4),
+    (128, 8, 48, 7, 4), (64, 48, 64, 8, 8), (192, 4, 24, 6, 4), (8, 64, 64, 8, 4),
+    (2, 65, 128, 10, 4), (4, 128, 256, 10, 8), (8, 200, 256, 10, 8), (12, 65, 256, 8, 3),
+    (8, 8, 130, 10, 4), (8, 256, 256, 12, 4),
 )
 
 
-def calibration_workload(B: int, lo: int, hi: int, *, H: int = 32, seed: int = 0):
-    """Synthetic batch of B frontier trees (depth ≤ 8, branching ≤ 4) whose sizes are
-    uniform in [lo, hi]; bf16 q / k / v, dk = dv = 128."""
+def calibration_workload(B: int, lo: int, hi: int, max_depth: int = 8, fmax: int = 4, *,
+                         H: int = 32, seed: int = 0):
+    """Synthetic batch of B frontier trees (paths up to ``max_depth`` deep, up to ``fmax``
+    children per node) whose sizes are uniform in [lo, hi]; bf16 q / k / v, dk = dv = 128."""
     from .workloads import frontier_tree, synthetic
-    rng = np.random.Generator(np.random.PCG64([seed, B, lo, hi]))
+    rng = np.random.Generator(np.random.PCG64([seed, B, lo, hi, max_depth, fmax]))
     sizes = [int(x) for x in rng.integers(lo, hi + 1, size=B)]
-    parents = [frontier_tree(int(rng.integers(1 << 30)), n, 8, 4)[0] for n in sizes]
+    parents = [frontier_tree(int(rng.integers(1 << 30)), n, max_depth, fmax)[0] for n in sizes]
     return synthetic(parents, H, 128, 128, seed=int(rng.integers(1 << 30)),
                      name=f"calib-B{B}-n{lo}..{hi}")
 
 
 def calibrate(H: int = 32, *, seed: int = 0, launches: int = 12,
-              batches: Sequence[Tuple[int, int, int]] = CALIBRATION_BATCHES
+              batches: Sequence[Tuple[int, int, int, int, int]] = CALIBRATION_BATCHES
               ) -> Tuple[CostModel, List[Tuple[List[int], int, float]]]:
     """Fit a `CostModel` on this GPU from `measure_us` of `calibration_workload` batches,
-    given as (B, smallest tree, largest tree).  Returns the model and its (sizes, H, µs)
-    samples."""
+    given as (B, smallest tree, largest tree, deepest path, most children).  Returns the
+    model and its (sizes, H, µs) samples."""
     import torch
     flush = torch.empty(64 << 20, dtype=torch.float32, device="cuda")
     samples = []
-    for B, lo, hi in batches:
-        w = calibration_workload(B, lo, hi, H=H, seed=seed)
+    for B, lo, hi, depth, fmax in batches:
+        w = calibration_workload(B, lo, hi, depth, fmax, H=H, seed=seed)
         us = measure_us(w, launches=launches, flush=flush)
         samples.append(([int(x) for x in np.diff(w.node_offsets)], H, us))
     return CostModel.fit(samples), samples

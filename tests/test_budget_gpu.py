@@ -18,7 +18,7 @@ def test_calibrated_model_predicts_unseen_batches():
         assert model.predict_us(sizes, H) == pytest.approx(us, rel=0.25)
     held_out = [W.config(3, 1), W.config(4, 1), W.config(5, 1),
                 Bd.calibration_workload(48, 20, 60, seed=9),
-                Bd.calibration_workload(6, 90, 220, seed=9)]
+                Bd.calibration_workload(6, 90, 220, 9, 6, seed=9)]
     for w in held_out:
         sizes = [int(x) for x in np.diff(w.node_offsets)]
         us = Bd.measure_us(w, launches=8)
