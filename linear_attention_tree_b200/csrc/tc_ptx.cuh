@@ -118,6 +118,10 @@ __device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
                "r"(bytes)
                : "memory");
 }
+// Prefetch the cache line holding `p` into L2.
+__device__ __forceinline__ void prefetch_line_l2(const void *p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)) : "memory");
+}
 // Prefetch one 3-D TMA box into L2 (nothing lands in shared memory).
 __device__ __forceinline__ void prefetch_tile_l2(const CUtensorMap *map, int x, int y, int z) {
   asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(

@@ -198,8 +198,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5;
   const int H = a.H;
   const int s = blockIdx.x / H, h = blockIdx.x % H, kh = qk_head(h, H, a.Hk);
-  // launched with programmatic stream serialisation: wait for the previous kernel before
-  // the first global access, and let the next one get its CTAs resident early
+  // Launched with programmatic stream serialisation: the kernel before this one on the
+  // stream may still be finishing.  Until it has (griddepcontrol.wait), this CTA only asks
+  // L2 for its S_root block and node range: a prefetch moves nothing into the CTA, and a
+  // write by that kernel to the same lines lands in L2 after it, so this is correct
+  // whatever it writes.  Then the kernel after this one may get its CTAs resident early.
+  if (threadIdx.x == 0) {
+    ptx::prefetch_l2(a.S_root + (size_t)blockIdx.x * 128 * 128, 128 * 128 * 4);
+    ptx::prefetch_line_l2(a.node_offsets + blockIdx.x / a.H);
+  }
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
