@@ -473,49 +473,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ptx::tc_fence_after();
 
-    // ---- 4. gamma o^T, R^T_c, zero U^T (lane v, node columns 32 ch .. 32 ch + 31) ----------
-    {
-      const int v = row, j0 = 32 * ch;
-      float o0[16], o1[16], k0[16], k1[16];
-      ptx::tmem_ld16(tlane + kColD + j0, o0);
-      ptx::tmem_ld16(tlane + kColD + j0 + 16, o1);
-      ptx::tmem_ld16(tlane + kColD + kTile + j0, k0);
-      ptx::tmem_ld16(tlane + kColD + kTile + j0 + 16, k1);
-      ptx::tmem_wait_ld();
+    // ---- 4 and 5 side by side: warps 4-7 form gamma o^T, R^T_c and U^T = 0 for all 64 node
+    // columns of their lanes (lane v = tid - 128) while warps 0-3 run the W rows (threads
+    // 0..63) and T rows (threads 64..127) of the tile's nodes.
+    if (tid >= 128) {
+      const int v = row;
       const unsigned char *vt = sm + kOffV + b * kKBytes + (v >> 6) * kKHalf + (v & 7) * 2;
       const int vc = (v & 63) >> 3;
+#pragma unroll 1
+      for (int j0 = 0; j0 < kTile; j0 += 32) {
+        float o0[16], o1[16], k0[16], k1[16];
+        ptx::tmem_ld16(tlane + kColD + j0, o0);
+        ptx::tmem_ld16(tlane + kColD + j0 + 16, o1);
+        ptx::tmem_ld16(tlane + kColD + kTile + j0, k0);
+        ptx::tmem_ld16(tlane + kColD + kTile + j0 + 16, k1);
+        ptx::tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int ja = j0 + j, jb = j0 + 16 + j;
-        o0[j] *= mt.gam[node0 + ja];
-        o1[j] *= mt.gam[node0 + jb];
-        const float va = __bfloat162float(
-            *reinterpret_cast<const __nv_bfloat16 *>(vt + ja * 128 + ((vc ^ (ja & 7)) << 4)));
-        const float vb = __bfloat162float(
-            *reinterpret_cast<const __nv_bfloat16 *>(vt + jb * 128 + ((vc ^ (jb & 7)) << 4)));
-        k0[j] = ja < nc ? tf32_rn(kGdn ? fmaf(-mt.bg[node0 + ja], k0[j], mt.bq[node0 + ja] * va) : va) : 0.f;
-        k1[j] = jb < nc ? tf32_rn(kGdn ? fmaf(-mt.bg[node0 + jb], k1[j], mt.bq[node0 + jb] * vb) : vb) : 0.f;
+        for (int j = 0; j < 16; ++j) {
+          const int ja = j0 + j, jb = j0 + 16 + j;
+          o0[j] *= mt.gam[node0 + ja];
+          o1[j] *= mt.gam[node0 + jb];
+          const float va = __bfloat162float(
+              *reinterpret_cast<const __nv_bfloat16 *>(vt + ja * 128 + ((vc ^ (ja & 7)) << 4)));
+          const float vb = __bfloat162float(
+              *reinterpret_cast<const __nv_bfloat16 *>(vt + jb * 128 + ((vc ^ (jb & 7)) << 4)));
+          k0[j] = ja < nc ? tf32_rn(kGdn ? fmaf(-mt.bg[node0 + ja], k0[j], mt.bq[node0 + ja] * va) : va) : 0.f;
+          k1[j] = jb < nc ? tf32_rn(kGdn ? fmaf(-mt.bg[node0 + jb], k1[j], mt.bq[node0 + jb] * vb) : vb) : 0.f;
+        }
+        ptx::tmem_st16(tlane + kColD + j0, o0);
+        ptx::tmem_st16(tlane + kColD + j0 + 16, o1);
+        ptx::tmem_st16(tlane + kColR + kTile * c + j0, k0);
+        ptx::tmem_st16(tlane + kColR + kTile * c + j0 + 16, k1);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) k0[j] = 0.f;
+        ptx::tmem_st16(tlane + kColD + kTile + j0, k0);
+        ptx::tmem_st16(tlane + kColD + kTile + j0 + 16, k0);
       }
-      ptx::tmem_st16(tlane + kColD + j0, o0);
-      ptx::tmem_st16(tlane + kColD + j0 + 16, o1);
-      ptx::tmem_st16(tlane + kColR + kTile * c + j0, k0);
-      ptx::tmem_st16(tlane + kColR + kTile * c + j0 + 16, k1);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) k0[j] = 0.f;
-      ptx::tmem_st16(tlane + kColD + kTile + j0, k0);
-      ptx::tmem_st16(tlane + kColD + kTile + j0 + 16, k0);
       ptx::tmem_wait_st();
+    } else if ((tid & 63) < nc) {
+      const int r = tid & 63, nn = node0 + r, d = mt.dep[nn];
+      if (tid < kTile) row_coefficients<true, kGdn>(mt, nn, r, d);
+      else row_coefficients<false, kGdn>(mt, nn, r, d);
     }
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    // ---- 5. W rows (threads 0..63) and T rows (threads 128..191) of this tile ---------------
-    if ((tid & 127) < kTile && (tid & 127) < nc) {
-      const int r = tid & 63, nn = node0 + r, d = mt.dep[nn];
-      if (tid < 128) row_coefficients<true, kGdn>(mt, nn, r, d);
-      else row_coefficients<false, kGdn>(mt, nn, r, d);
-    }
-    __syncthreads();
 
     // ---- 6. path MMAs, one coefficient block per tile c' holding path nodes -----------------
     for (int c2 = 0; c2 <= c; ++c2) {
