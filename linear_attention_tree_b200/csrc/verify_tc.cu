@@ -19,8 +19,10 @@
 //
 // The accumulator is kept transposed -- tensor-memory lane = value index, column = node --
 // so that R^T can be formed in place and fed back to the tensor core from tensor memory,
-// and so that every warp's output store is a contiguous 128-byte row segment.
+// and so that every lane holds one value index of a node's output row.
 // Order of work in one CTA (one item; two CTAs per SM):
+//   0. before the previous kernel on the stream has completed: an L2 prefetch of the
+//      item's S_root block and node range only.
 //   1. the S_root loads (64 KiB) go out first, into registers; TMA brings q, k, v in the
 //      128-byte swizzled layout the MMA reads.
 //   2. Gram MMA (tcgen05 kind::f16, 128 x 64 x 128): [Q ; K] . K^T into columns 128..191,
@@ -32,8 +34,11 @@
 //      b_j gamma_j (S_root k_j)[v] into columns 192..255 (tf32); [W ; T] written as the
 //      shared-memory operand.
 //   7. path-sum MMA (kind::tf32, A = R^T from tensor memory): columns 0..127 (o part
-//      rescaled, U part zeroed in step 6) += R^T . [W ; T]^T, i.e. o^T and U^T.
-//   8. tensor memory -> registers -> 128-byte row segments of o and U.
+//      rescaled, U part zeroed in step 6) += R^T . [W ; T]^T, i.e. o^T and U^T, as two
+//      N = 64 chains (W -> o, T -> U) issued by two threads.
+//   8. tensor memory -> registers; a full tree's o and U node rows go through shared
+//      memory and leave by one TMA tensor store each, a smaller tree's as 128-byte row
+//      segments per warp.
 // Trees deeper than kRegDepth take dense Gram matrices and an in-shared-memory recursion
 // in step 6 instead of steps 3-4.
 //

@@ -13,29 +13,36 @@
 // a 4-word ancestor bitmask, word c' holds exactly the path nodes that lie in tile c'.
 // One CTA of 256 threads per (sequence, head), one CTA per SM:
 //   0. TMA: S_root (four 32-column fp32 chunks) and the q / k / v tiles of tiles 0 and 1.
-//      Tree walk (one thread per node): ancestor bits, depth, root-first paths, cl, gamma.
+//      Tree walk (one thread per node): ancestor bits, depth, root-first paths, cl, gamma,
+//      and per tile the set of tiles holding path nodes of its nodes (warp OR-reductions).
 //   1. S_root fp32 -> bf16, row v into tensor-memory lane v (the state MMA's A operand);
 //      then the k tiles of tiles 0..N/64-2 into the freed staging area, where the Gram
 //      blocks of later tiles read them.
 //   for every tile c:
 //   2. Gram blocks [Q_c ; K_c] . K_c'^T (tcgen05 kind::f16) for every c' <= c in one batch:
 //      the earlier tiles' k rows lie back to back in shared memory, so they form one operand
-//      of 64 c rows (one MMA chain, N = 64 c), and the tile's own k rows another (N = 64).
-//      The entries are stored by path position: q_n.k_i for i on path(n) (this tile's rows),
-//      b_n k_n.k_i for i in anc(n) (kept for all nodes).
+//      of 64 c rows (one MMA chain, N = 64 c), and the tile's own k rows another (N = 64);
+//      three threads issue the chains.  Each thread stages its row's 32 values of a block in
+//      shared memory and picks out its path columns: q_n.k_i for i on path(n) (this tile's
+//      rows), b_n k_n.k_i for i in anc(n) (kept for all nodes), stored by path position.
 //   3. state MMA S_root . [Q_c ; K_c]^T (kind::f16, A = S_root from tensor memory), in the
 //      same batch as the Gram chains when their columns do not overlap its own.
-//   4. per value lane: o columns scaled by gamma_n, R^T_c[v][j] = b_j v_j[v] - b_j gamma_j
-//      (S_root k_j)[v] (tf32) into tensor memory next to the R^T of earlier tiles, U zeroed.
-//   5. T and W rows of the tile's nodes (register recursions, paths up to kDepth deep).
-//   6. path MMAs, one per tile c' <= c holding path nodes: [o ; U]_c^T += R^T_c' . [W ; T]_c,c'^T
-//      (kind::tf32, A = R^T_c' from tensor memory, B = the coefficient block in shared memory).
-//   7. o_c and U_c from tensor memory to 128-byte row segments.
+//   4. warps 4-7, per value lane and all 64 node columns: o columns scaled by gamma_n,
+//      R^T_c[v][j] = b_j v_j[v] - b_j gamma_j (S_root k_j)[v] (tf32) into tensor memory next
+//      to the R^T of earlier tiles, U zeroed; meanwhile warps 0-3 run the T and W rows of
+//      the tile's nodes (register recursions, paths up to kDepth deep).
+//   5. path MMAs, one per tile c' <= c holding path nodes: [o ; U]_c^T += R^T_c' . [W ; T]_c,c'^T
+//      (kind::tf32, A = R^T_c' from tensor memory, B = the coefficient block in shared
+//      memory, built from each row's path positions in tile c'; two N = 64 chains).
+//   6. o_c and U_c from tensor memory: a full tile as node rows in shared memory and two TMA
+//      tensor stores (read out before the next tile's extraction, after which that buffer
+//      takes the tile two ahead), a ragged last tile as 128-byte row segments.
 // Tensor memory (512 columns): [0, 256) R^T of the four tiles, [256, 384) o^T | U^T of the
 // current tile, [384, 448) S_root in bf16, [448, 512) the Gram block of the tile's own k rows.
 // The Gram blocks of tile c against tiles 0..c-1 go to [64 c, 128 c): R^T columns of tiles
 // c.. (written later, in step 4) and, for c = 3, the o^T | U^T columns (the state MMA then
-// waits until they are read).
+// waits until they are read).  Shared memory holds two q / k / v buffers (tile c in buffer
+// c & 1), one coefficient buffer and the k rows of tiles 0..2.
 // Trees deeper than kDepth are verified by the CUDA-core algorithm in the same CTA.
 //
 // Every wait is bounded: a wait that runs out records TV_ERR_TIMEOUT on the status word; the
@@ -473,9 +480,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ptx::tc_fence_after();
 
-    // ---- 4 and 5 side by side: warps 4-7 form gamma o^T, R^T_c and U^T = 0 for all 64 node
-    // columns of their lanes (lane v = tid - 128) while warps 0-3 run the W rows (threads
-    // 0..63) and T rows (threads 64..127) of the tile's nodes.
+    // ---- 4. warps 4-7 form gamma o^T, R^T_c and U^T = 0 for all 64 node columns of their
+    // lanes (lane v = tid - 128) while warps 0-3 run the W rows (threads 0..63) and T rows
+    // (threads 64..127) of the tile's nodes.
     if (tid >= 128) {
       const int v = row;
       const unsigned char *vt = sm + kOffV + b * kKBytes + (v >> 6) * kKHalf + (v & 7) * 2;
@@ -519,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
 
-    // ---- 6. path MMAs, one coefficient block per tile c' holding path nodes -----------------
+    // ---- 5. path MMAs, one coefficient block per tile c' holding path nodes -----------------
     for (int c2 = 0; c2 <= c; ++c2) {
       if (!((blkm >> c2) & 1u)) continue;
       {
@@ -567,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ptx::tc_fence_after();
 
-    // ---- 7. o_c and U_c (lane v, node columns 32 ch .. 32 ch + 31) --------------------------
+    // ---- 6. o_c and U_c (lane v, node columns 32 ch .. 32 ch + 31) --------------------------
     {
       const int v = row, j0 = 32 * ch;
       float o0[16], o1[16], u0[16], u1[16];
