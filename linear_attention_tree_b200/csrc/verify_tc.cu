@@ -21,8 +21,8 @@
 // so that R^T can be formed in place and fed back to the tensor core from tensor memory,
 // and so that every lane holds one value index of a node's output row.
 // Order of work in one CTA (one item; two CTAs per SM):
-//   0. before the previous kernel on the stream has completed: an L2 prefetch of the
-//      item's S_root block and node range only.
+//   0. before the previous kernel on the stream has completed (first resident wave): an L2
+//      prefetch of the item's S_root block and node range only.
 //   1. the S_root loads (64 KiB) go out first, into registers; TMA brings q, k, v in the
 //      128-byte swizzled layout the MMA reads.
 //   2. Gram MMA (tcgen05 kind::f16, 128 x 64 x 128): [Q ; K] . K^T into columns 128..191,
@@ -348,11 +348,13 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int H = a.H;
   const int s = blockIdx.x / H, h = blockIdx.x % H, kh = qk_head(h, H, a.Hk);
   // Launched with programmatic stream serialisation: the kernel before this one on the
-  // stream may still be finishing.  Until it has (griddepcontrol.wait), this CTA only asks
-  // L2 for its S_root block and node range: a prefetch moves nothing into the CTA, and a
-  // write by that kernel to the same lines lands in L2 after it, so this is correct
-  // whatever it writes.  Then the kernel after this one may get its CTAs resident early.
-  if (threadIdx.x == 0) {
+  // stream may still be finishing.  Until it has (griddepcontrol.wait), a CTA of the first
+  // resident wave only asks L2 for its S_root block and node range: a prefetch moves
+  // nothing into the CTA, and a write by that kernel to the same lines lands in L2 after
+  // it, so this is correct whatever it writes (later waves start after that kernel is done
+  // and have their blocks prefetched by the wave before).  Then the kernel after this one
+  // may get its CTAs resident early.
+  if (threadIdx.x == 0 && (int)blockIdx.x < prefetch_stride) {
     ptx::prefetch_l2(a.S_root + (size_t)blockIdx.x * 128 * 128, 128 * 128 * 4);
     ptx::prefetch_line_l2(a.node_offsets + blockIdx.x / a.H);
   }
