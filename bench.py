@@ -517,7 +517,10 @@ def run_b200(args, workloads):
         if world == 1 and not args.other_configs_off:
             line["other_workloads"] = other_workloads(args, L, dev, peak)
         if world == 1 and not args.no_budget:
-            line["batch_budget"] = batch_budget(line, 1e6 * c_avg)
+            try:
+                line["batch_budget"] = batch_budget(line, 1e6 * c_avg)
+            except Exception as e:   # an auxiliary figure: report it, keep the line
+                line["batch_budget"] = {"error": f"{type(e).__name__}: {e}"}
         if world == 1 and not args.no_cpu_baseline:
             got = tuple(t.float().cpu().numpy().astype(np.float64) for t in outs[0])
             line["cpu_baseline"] = cpu_baseline_and_self_check(workloads[0], got)
