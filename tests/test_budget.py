@@ -221,3 +221,22 @@ def test_time_budget_and_chosen_budget_match_an_exhaustive_scan():
     small = Bd.choose_budget(trees, 32, model, fixed_us=0.0)["budget"]
     large = Bd.choose_budget(trees, 32, model, fixed_us=2000.0)["budget"]
     assert large >= small
+
+
+def test_edge_cases():
+    assert Bd.select_nodes([], 5) == []
+    assert [len(k) for k in Bd.select_nodes([([], [])], 5)] == [0]
+    # equal (zero) probabilities: the shallower node first, then the next tree
+    keeps = Bd.select_nodes([([-1, 0], [0.0, 0.0]), ([-1], [1.0])], 2)
+    assert [list(k) for k in keeps] == [[0], [0]]
+    assert [len(k) for k in Bd.select_nodes([([-1, 0, 0], [0.5] * 3)], 3, cap=0)] == [0]
+    # a reserve larger than a tree keeps the whole tree
+    assert [list(k) for k in Bd.select_nodes([([-1, 0], [0.5, 0.5])], 2, min_nodes=5)] == [[0, 1]]
+    assert list(Bd.cap_largest([], 3)) == [] and list(Bd.cap_largest([3, 3], 0)) == [0, 0]
+    par, offs, rows = Bd.pack([], [])
+    assert len(par) == 0 and list(offs) == [0] and len(rows) == 0
+    assert Bd.B200_DEFAULT.predict_us([], 32) == pytest.approx(Bd.B200_DEFAULT.tc[0])
+    with pytest.raises(ValueError):
+        Bd.allocate_time([([-1, 0], [0.5, 0.5])], 32, 1.0)
+    with pytest.raises(ValueError):
+        Bd.select_nodes([([-1], [0.5])], -1)
