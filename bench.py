@@ -480,6 +480,8 @@ def run_b200(args, workloads):
                          "algorithmic_bytes_per_launch": vb,
                          "frac_of_8TBps": achieved / NOMINAL_HBM_GBS},
             "verify_us": 1e6 * v_avg, "commit_us": 1e6 * c_avg,
+            "verify_us_p10_p50_p90": [1e3 * float(np.percentile(verify_ms, q)) for q in (10, 50, 90)],
+            "commit_us_p10_p50_p90": [1e3 * float(np.percentile(commit_ms, q)) for q in (10, 50, 90)],
             "kernel_timing": f"events around each kernel, second timed pass of {k_steps} steps",
             "verify_nodes_per_s": T / v_avg,
             "commit_roofline": {"achieved": cb / c_avg / 1e9, "unit": "GB/s",
