@@ -414,6 +414,62 @@ def test_p10_single_token():
 
 
 # ------------------------------------------------------------------------- metadata, commit
+def _hadamard16():
+    h = np.array([[1.0]])
+    for _ in range(4):
+        h = np.block([[h, h], [h, -h]])
+    return h / 4.0          # orthonormal rows, every entry +-1/4 (exact in fp32)
+
+
+def pin_orthonormal_keys(seed=43):
+    """Gated delta rule with mutually orthonormal keys along every path (general a, b).
+
+    The factors (I - b_i k_i k_i^T) of orthonormal keys commute and each k_i passes through
+    the others unchanged, so the recurrence closes to
+        S_n = gamma_n S_root (I - sum_i b_i k_i k_i^T) + sum_i exp(cl_n - cl_i) b_i v_i k_i^T,
+        u_n = b_n (v_n - gamma_n S_root k_n)        (the tree system's L vanishes: U = R),
+    sums over path(n), cl the path sum of log_a and gamma = exp(cl).
+    """
+    rng = np.random.default_rng(seed)
+    for trial in range(4):
+        n = int(rng.integers(2, 15))
+        par = W.uniform_parent_tree(rng, n, 6)
+        w = W.synthetic([par], H=2, dk=16, dv=5, seed=seed * 100 + trial, in_dtype="f32",
+                        log_a_mean=-1.0)
+        for h in range(2):
+            rows = rng.permutation(16)[:n]
+            signs = rng.choice([-1.0, 1.0], size=n)
+            w.k[:, h, :] = (_hadamard16()[rows] * signs[:, None]).astype(np.float32)
+        dk = 16
+        for h in range(2):
+            S0 = w.S_root[0, h].astype(np.float64)
+            k, v = w.k[:, h].astype(np.float64), w.v[:, h].astype(np.float64)
+            la, b = w.log_a[:, h].astype(np.float64), w.b[:, h].astype(np.float64)
+            S = O.node_states(w, 0, h)
+            for node in range(n):
+                path = []
+                x = node
+                while x >= 0:
+                    path.append(x)
+                    x = par[x]
+                path.reverse()
+                cl = np.cumsum(la[path])
+                proj = np.eye(dk) - sum(b[i] * np.outer(k[i], k[i]) for i in path)
+                want = np.exp(cl[-1]) * S0 @ proj
+                for j, i in enumerate(path):
+                    want = want + np.exp(cl[-1] - cl[j]) * b[i] * np.outer(v[i], k[i])
+                np.testing.assert_allclose(S[node], want, rtol=1e-10, atol=1e-12)
+                o, u = O.verify_node(w, 0, node, h)
+                np.testing.assert_allclose(u, b[node] * (v[node] - np.exp(cl[-1]) * S0 @ k[node]),
+                                           rtol=1e-10, atol=1e-12)
+                np.testing.assert_allclose(o, want @ w.q[node, h].astype(np.float64),
+                                           rtol=1e-10, atol=1e-12)
+
+
+def test_p11_orthonormal_keys():
+    pin_orthonormal_keys()
+
+
 def test_meta_worked_example():
     w = W.config(1)
     depth, anc, cl = O.tree_meta(w.parent, w.log_a)
@@ -520,7 +576,8 @@ def test_commit_empty_path_is_root_and_matches_node_states():
 
 # ------------------------------------------------------------------------ planted mistakes
 _PINS = [pin_worked_example, pin_closed_form_scalar, pin_chain_is_sequential, pin_b_zero,
-         pin_delta_rule, lambda: pin_bruteforce(max_n=4), pin_lossless_wy, pin_single_token]
+         pin_delta_rule, lambda: pin_bruteforce(max_n=4), pin_lossless_wy, pin_single_token,
+         pin_orthonormal_keys]
 
 _orig_step = O.step
 _orig_verify_node = O.verify_node
