@@ -97,16 +97,9 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t sr
                "r"(src), "r"(x), "r"(y), "r"(z)
                : "memory");
 }
-// Contiguous shared -> global bulk copy (addresses 16-byte aligned, bytes a multiple of 16),
-// tracked by this thread's bulk groups; commit_group closes a group, wait_group_read waits
-// until the thread's groups have finished reading shared memory, wait_group until they
-// have completed.
-__device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
-                   reinterpret_cast<uint64_t>(dst)),
-               "r"(src), "r"(bytes)
-               : "memory");
-}
+// Bulk groups of this thread's asynchronous shared -> global copies (TMA stores):
+// commit_group closes a group, wait_group_read waits until the thread's groups have finished
+// reading shared memory, wait_group until they have completed.
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
