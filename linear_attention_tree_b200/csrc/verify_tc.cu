@@ -137,8 +137,12 @@ __device__ __forceinline__ float4 ldg_first(const float4 *p) {
                : "l"(p));
   return r;
 }
-__device__ __forceinline__ void st_out(float *p, float x) { __stcs(p, x); }
-__device__ __forceinline__ void st_out(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
+// Tensor maps over the output rows [T][H][128] with boxes of 64, 32, 16, 8, 4, 2 and 1 node
+// rows: a tree of n nodes leaves by one tensor store per set bit of n.
+constexpr int kRowMaps = 7;
+struct RowMaps {
+  CUtensorMap m[kRowMaps];
+};
 
 // One K = 128 chain of bf16 MMAs: D = A . B^T with A and B 128-row K-major operands.
 __device__ __forceinline__ void mma_chain_bf16(uint32_t a_base, uint32_t b_base, uint32_t d_tmem,
@@ -336,8 +340,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     verify_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v,
-                     const __grid_constant__ CUtensorMap tm_o,
-                     const __grid_constant__ CUtensorMap tm_u, VerifyArgs a, FuseArgs f,
+                     const __grid_constant__ RowMaps tm_o,
+                     const __grid_constant__ RowMaps tm_u, VerifyArgs a, FuseArgs f,
                      int prefetch_stride) {
   extern __shared__ unsigned char smem_dyn[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
@@ -722,57 +726,45 @@ __global__ void __launch_bounds__(kThreads, 2)
     ptx::tmem_ld16(tlane + kTile + j0 + 16, u1);
     ptx::tmem_wait_ld();
     release_tmem(warp, tmem);
-    if (n_nodes == kTile) {
-      // a full tree: node rows into shared memory (o over the dead [W ; T] operand, U over
-      // the dead S_root operand), then one tensor store each; the CTA leaves once they have
-      // been read out of shared memory
-      Tout *ost = reinterpret_cast<Tout *>(sm + kOffA2);
+    // node rows into shared memory (o over the dead [W ; T] operand, U over the dead S_root
+    // operand), then tensor stores of 64, 32, ..., 1 rows, one per set bit of n_nodes; the
+    // CTA leaves once they have been read out of shared memory
+    Tout *ost = reinterpret_cast<Tout *>(sm + kOffA2);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      ost[(j0 + j) * 128 + v] = from_f32<Tout>(o0[j]);
+      ost[(j0 + 16 + j) * 128 + v] = from_f32<Tout>(o1[j]);
+    }
+    if (a.u_bf16) {
+      __nv_bfloat16 *ust = reinterpret_cast<__nv_bfloat16 *>(sm + kOffS);
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        ost[(j0 + j) * 128 + v] = from_f32<Tout>(o0[j]);
-        ost[(j0 + 16 + j) * 128 + v] = from_f32<Tout>(o1[j]);
-      }
-      if (a.u_bf16) {
-        __nv_bfloat16 *ust = reinterpret_cast<__nv_bfloat16 *>(sm + kOffS);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          ust[(j0 + j) * 128 + v] = __float2bfloat16_rn(u0[j]);
-          ust[(j0 + 16 + j) * 128 + v] = __float2bfloat16_rn(u1[j]);
-        }
-      } else {
-        float *ust = reinterpret_cast<float *>(sm + kOffS);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          ust[(j0 + j) * 128 + v] = u0[j];
-          ust[(j0 + 16 + j) * 128 + v] = u1[j];
-        }
-      }
-      ptx::fence_proxy_async_smem();
-      __syncthreads();
-      if (tid == 0) {
-        ptx::tma_store_3d(&tm_o, sbase + kOffA2, 0, h, lo);
-        ptx::tma_store_3d(&tm_u, sbase + kOffS, 0, h, lo);
-        ptx::bulk_commit();
-        ptx::bulk_wait_read();
+        ust[(j0 + j) * 128 + v] = __float2bfloat16_rn(u0[j]);
+        ust[(j0 + 16 + j) * 128 + v] = __float2bfloat16_rn(u1[j]);
       }
     } else {
-      Tout *out = static_cast<Tout *>(a.out) + ((size_t)lo * H + h) * 128 + v;
-      const size_t ub = ((size_t)lo * H + h) * 128 + v;
-      const size_t rs = (size_t)H * 128;
+      float *ust = reinterpret_cast<float *>(sm + kOffS);
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        if (j0 + j < n_nodes) {
-          st_out(out + (j0 + j) * rs, o0[j]);
-          store_u(a.U, ub + (j0 + j) * rs, u0[j], a.u_bf16);
+        ust[(j0 + j) * 128 + v] = u0[j];
+        ust[(j0 + 16 + j) * 128 + v] = u1[j];
+      }
+    }
+    ptx::fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      const uint32_t orow = 128 * sizeof(Tout), urow = a.u_bf16 ? 256u : 512u;
+      int j = 0;
+      for (int i = 0; i < kRowMaps; ++i) {
+        const int r = kTile >> i;
+        if (n_nodes & r) {
+          ptx::tma_store_3d(&tm_o.m[i], sbase + kOffA2 + j * orow, 0, h, lo + j);
+          ptx::tma_store_3d(&tm_u.m[i], sbase + kOffS + j * urow, 0, h, lo + j);
+          j += r;
         }
       }
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        if (j0 + 16 + j < n_nodes) {
-          st_out(out + (j0 + 16 + j) * rs, o1[j]);
-          store_u(a.U, ub + (j0 + 16 + j) * rs, u1[j], a.u_bf16);
-        }
-      }
+      ptx::bulk_commit();
+      ptx::bulk_wait_read();
     }
   }
 }
@@ -780,15 +772,18 @@ __global__ void __launch_bounds__(kThreads, 2)
 // ---- host side ------------------------------------------------------------------------
 template <bool kGdn, typename Tout, bool kFused>
 cudaError_t launch_tc_t(const VerifyArgs &a, const FuseArgs &f, cudaStream_t st) {
-  CUtensorMap mq, mk, mv, mo, mu;
+  CUtensorMap mq, mk, mv;
+  RowMaps mo, mu;
   // (a next tree with no nodes at all still gets maps over a one-row view: the kernel only
   // commits then)
   const int rows = a.T > 0 ? a.T : 1;
   if (!make_node_map(&mq, a.q, a.Hk, rows, kTile) || !make_node_map(&mk, a.k, a.Hk, rows, kTile) ||
-      !make_node_map(&mv, a.v, a.H, rows, kTile) ||
-      !make_row_map(&mo, a.out, sizeof(Tout) == 2, a.H, rows, kTile) ||
-      !make_row_map(&mu, a.U, a.u_bf16 != 0, a.H, rows, kTile))
+      !make_node_map(&mv, a.v, a.H, rows, kTile))
     return cudaErrorInvalidValue;
+  for (int i = 0; i < kRowMaps; ++i)
+    if (!make_row_map(&mo.m[i], a.out, sizeof(Tout) == 2, a.H, rows, kTile >> i) ||
+        !make_row_map(&mu.m[i], a.U, a.u_bf16 != 0, a.H, rows, kTile >> i))
+      return cudaErrorInvalidValue;
   auto kern = verify_tc_kernel<kGdn, Tout, kFused>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
