@@ -36,9 +36,8 @@
 //   7. path-sum MMA (kind::tf32, A = R^T from tensor memory): columns 0..127 (o part
 //      rescaled, U part zeroed in step 6) += R^T . [W ; T]^T, i.e. o^T and U^T, as two
 //      N = 64 chains (W -> o, T -> U) issued by two threads.
-//   8. tensor memory -> registers; a full tree's o and U node rows go through shared
-//      memory and leave by one TMA tensor store each, a smaller tree's as 128-byte row
-//      segments per warp.
+//   8. tensor memory -> registers -> o and U node rows in shared memory -> TMA tensor
+//      stores of 64, 32, ..., 1 rows, one per set bit of the tree's size.
 // Trees deeper than kRegDepth take dense Gram matrices and an in-shared-memory recursion
 // in step 6 instead of steps 3-4.
 //
@@ -716,7 +715,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
   ptx::tc_fence_after();
 
-  // ---- 8. o^T and U^T -> 128-byte row segments (a warp's 32 lanes are 32 adjacent v) -----
+  // ---- 8. o^T and U^T -> node rows in shared memory (a warp's 32 lanes are 32 adjacent v) --
   {
     const int v = quarter * 32 + lane, j0 = set * 32;
     float o0[16], o1[16], u0[16], u1[16];
